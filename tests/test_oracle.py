@@ -1,0 +1,337 @@
+"""Pins for the oracle: each test checks it against something other than its
+own code -- brute force on tiny inputs, a library routine (torch SDPA in fp64),
+closed forms, the pages' invariants and the numbers the pages print."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import krea_oracle as ko
+from synth.inputs import Case, make_inputs, tiny_dense
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def f64(t):
+    return t.double().numpy()
+
+
+def small_case(mode="dense", **kw):
+    base = dict(name="s", batch=1, q_heads=8, kv_heads=2, head_dim=64, text_len=40, grid_h=12, grid_w=12,
+                dtype="f16", mode=mode, seed=11)
+    base.update(kw)
+    return Case(**base)
+
+
+def token_rule_mask(T, H, W, window):
+    """Admission by the scanline token rule, written from the page: text tokens see
+    everything and are seen by everyone; an image token sees image tokens whose grid
+    row is at most window // 2 away."""
+    L = T + H * W
+    m = np.zeros((L, L), dtype=bool)
+    row = [None] * T + [i // W for i in range(H * W)]
+    for a in range(L):
+        for b in range(L):
+            if a < T or b < T:
+                m[a, b] = True
+            else:
+                m[a, b] = abs(row[a] - row[b]) <= window // 2
+    return m
+
+
+# --------------------------------------------------------------------------- brute force
+
+def brute_force(q, k, v, gate, scale, allowed):
+    """Per (head, row) loops over keys with math.exp, K/V expanded by repeat_interleave."""
+    B, L, Hq, d = q.shape
+    rep = Hq // k.shape[2]
+    ke = np.repeat(k, rep, axis=2)  # repeat_interleave order: head h -> kv head h // rep
+    ve = np.repeat(v, rep, axis=2)
+    out = np.zeros_like(q)
+    for b in range(B):
+        for h in range(Hq):
+            for t in range(L):
+                keys = [j for j in range(L) if allowed[t, j]]
+                s = [scale * float(np.dot(q[b, t, h], ke[b, j, h])) for j in keys]
+                mx = max(s)
+                w = [math.exp(x - mx) for x in s]
+                z = sum(w)
+                o = sum(wi / z * ve[b, j, h] for wi, j in zip(w, keys))
+                if gate is not None:
+                    o = o / (1.0 + np.exp(-gate[b, t, h]))
+                out[b, t, h] = o
+    return out
+
+
+def test_brute_force_tiny_dense():
+    c = tiny_dense()
+    q, k, v, _ = make_inputs(c)
+    ref = ko.attention(c, q, k, v)["out"]
+    L = c.seq_len
+    bf = brute_force(f64(q), f64(k), f64(v), None, 1 / 8, np.ones((L, L), bool))
+    assert np.max(np.abs(ref - bf)) < 1e-12
+
+
+def test_brute_force_scanline_token_rule_with_gate():
+    c = small_case("scanline", text_len=20, grid_h=6, grid_w=7, window=3, tile_aligned=False,
+                   q_heads=4, kv_heads=2, gate=True)
+    q, k, v, g = make_inputs(c)
+    ref = ko.attention(c, q, k, v, g)["out"]
+    allowed = token_rule_mask(c.text_len, c.grid_h, c.grid_w, c.window)
+    bf = brute_force(f64(q), f64(k), f64(v), f64(g), 1 / math.sqrt(64), allowed)
+    assert np.max(np.abs(ref - bf)) < 1e-12
+
+
+# --------------------------------------------------------------------------- library routine
+
+def sdpa_ref(q, k, v, mask, scale):
+    """torch.nn.functional.scaled_dot_product_attention in fp64 with expanded K/V."""
+    rep = q.shape[2] // k.shape[2]
+    qt = q.double().permute(0, 2, 1, 3)
+    kt = k.double().repeat_interleave(rep, dim=2).permute(0, 2, 1, 3)
+    vt = v.double().repeat_interleave(rep, dim=2).permute(0, 2, 1, 3)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=torch.from_numpy(mask),
+                                                          scale=scale)
+    return o.permute(0, 2, 1, 3).numpy()
+
+
+def test_dense_equals_sdpa():
+    c = small_case("dense", batch=2)
+    q, k, v, _ = make_inputs(c)
+    ref = ko.attention(c, q, k, v)["out"]
+    L = c.seq_len
+    lib = sdpa_ref(q, k, v, np.ones((L, L), bool), 1 / 8)
+    assert np.max(np.abs(ref - lib)) < 1e-10
+
+
+def test_scanline_token_rule_equals_masked_sdpa():
+    c = small_case("scanline", window=5, tile_aligned=False, grid_h=14, grid_w=11, text_len=77)
+    q, k, v, _ = make_inputs(c)
+    ref = ko.attention(c, q, k, v)["out"]
+    lib = sdpa_ref(q, k, v, token_rule_mask(c.text_len, c.grid_h, c.grid_w, c.window), 1 / 8)
+    assert np.max(np.abs(ref - lib)) < 1e-10
+
+
+def test_scanline_tile_aligned_equals_sdpa_on_active_tiles():
+    # tile_aligned: a pair is admitted iff both tokens are real and their logical
+    # 128-slot tiles form an active tile pair (one holding a pair the rule admits)
+    T, H, W, win = 200, 24, 20, 3
+    c = small_case("scanline", window=win, tile_aligned=True, grid_h=H, grid_w=W, text_len=T)
+    q, k, v, _ = make_inputs(c)
+    ref = ko.attention(c, q, k, v)["out"]
+    rule = token_rule_mask(T, H, W, win)
+    Pt = 512
+    slot = np.array([t if t < T else Pt + t - T for t in range(T + H * W)])
+    tile = slot // 128
+    nt = tile.max() + 1
+    active = np.zeros((nt, nt), bool)
+    for a in range(T + H * W):
+        for b in np.nonzero(rule[a])[0]:
+            active[tile[a], tile[b]] = True
+    mask = active[tile[:, None], tile[None, :]]
+    lib = sdpa_ref(q, k, v, mask, 1 / 8)
+    assert np.max(np.abs(ref - lib)) < 1e-10
+
+
+# --------------------------------------------------------------------------- closed forms
+
+def _q_zero_case(**kw):
+    c = small_case(**kw)
+    q, k, v, _ = make_inputs(c)
+    L = c.seq_len
+    q = torch.zeros_like(q)
+    vv = torch.zeros_like(v)
+    vv[..., 0] = 1.0
+    vv[..., 1] = torch.arange(L, dtype=torch.float64).to(v.dtype)[None, :, None]  # exact up to 2048 in f16
+    return c, q, k, vv
+
+
+def test_q_zero_gives_mean_of_admitted_values_dense():
+    c, q, k, v = _q_zero_case(mode="dense")
+    out = ko.attention(c, q, k, v)["out"]
+    L = c.seq_len
+    assert np.allclose(out[..., 0], 1.0, atol=1e-13)
+    assert np.allclose(out[..., 1], (L - 1) / 2, atol=1e-10)
+
+
+def test_q_zero_scanline_window_closed_form():
+    T, H, W, win = 30, 9, 10, 3
+    c, q, k, v = _q_zero_case(mode="scanline", text_len=T, grid_h=H, grid_w=W, window=win,
+                              tile_aligned=False)
+    out = ko.attention(c, q, k, v)["out"][0, :, 0, 1]
+    L = T + H * W
+    for t in range(L):
+        if t < T:
+            expect = (L - 1) / 2
+        else:
+            r = (t - T) // W
+            rows = range(max(0, r - win // 2), min(H, r + win // 2 + 1))
+            idx = list(range(T)) + [T + rr * W + cc for rr in rows for cc in range(W)]
+            expect = sum(idx) / len(idx)
+        assert abs(out[t] - expect) < 1e-9, t
+
+
+def test_constant_values_and_gate():
+    c = small_case("dense", gate=True)
+    q, k, v, g = make_inputs(c)
+    v = torch.full_like(v, 0.75)
+    out = ko.attention(c, q, k, v, g)["out"]
+    sig = 1 / (1 + np.exp(-f64(g)))
+    assert np.max(np.abs(out - 0.75 * sig)) < 1e-12
+    g0 = torch.zeros_like(g)
+    out0 = ko.attention(c, q, k, v, g0)["out"]
+    assert np.max(np.abs(out0 - 0.375)) < 1e-12
+
+
+def test_dominant_key():
+    c = small_case("dense", text_len=8, grid_h=4, grid_w=4, q_heads=2, kv_heads=1)
+    q, k, v, _ = make_inputs(c)
+    qd = f64(q)
+    j = 13
+    qd[0, 5, 0] = 40.0 * f64(k)[0, j, 0]
+    out = ko.attention(c, torch.from_numpy(qd), k, v)["out"]
+    assert np.max(np.abs(out[0, 5, 0] - f64(v)[0, j, 0])) < 1e-6
+
+
+def test_gqa_equals_explicit_expansion():
+    c = small_case("dense", q_heads=8, kv_heads=2)
+    q, k, v, _ = make_inputs(c)
+    out = ko.attention(c, q, k, v)["out"]
+    ce = small_case("dense", q_heads=8, kv_heads=8)
+    out_e = ko.attention(ce, q, k.repeat_interleave(4, dim=2), v.repeat_interleave(4, dim=2))["out"]
+    assert np.max(np.abs(out - out_e)) < 1e-13
+
+
+def test_probabilities_rows_sum_to_one_masked_zero():
+    c = small_case("scanline", window=3, tile_aligned=False, text_len=20, grid_h=6, grid_w=9)
+    q, k, v, _ = make_inputs(c)
+    P = ko.attention(c, q, k, v, return_probs=True)["probs"]
+    assert np.allclose(P.sum(-1), 1.0, atol=1e-13)
+    allowed = token_rule_mask(c.text_len, c.grid_h, c.grid_w, c.window)
+    assert np.all(P[:, :, ~allowed] == 0.0)
+    assert np.all(P[:, :, allowed] > 0.0)
+
+
+# --------------------------------------------------------------------------- invariants
+
+def test_wide_window_equals_dense():
+    T, H, W = 50, 7, 13
+    for ta in (True, False):
+        c = small_case("scanline", text_len=T, grid_h=H, grid_w=W, window=2 * H - 1, tile_aligned=ta)
+        q, k, v, _ = make_inputs(c)
+        out = ko.attention(c, q, k, v)["out"]
+        cd = small_case("dense", text_len=T, grid_h=H, grid_w=W)
+        outd = ko.attention(cd, q, k, v)["out"]
+        assert np.max(np.abs(out - outd)) < 1e-12
+
+
+def test_smooth_k_is_exact_for_fp16_tiles():
+    c = small_case("tilemix", pattern="zero", smooth_k=True, qk_dist="normal_koffset")
+    q, k, v, _ = make_inputs(c)
+    on = ko.attention(c, q, k, v)["out"]
+    c.smooth_k = False
+    off = ko.attention(c, q, k, v)["out"]
+    assert np.max(np.abs(on - off)) < 1e-12
+
+
+def test_pattern_zero_equals_dense():
+    c = small_case("tilemix", pattern="zero")
+    q, k, v, _ = make_inputs(c)
+    a = ko.attention(c, q, k, v)["out"]
+    b = ko.attention(small_case("dense"), q, k, v)["out"]
+    assert np.max(np.abs(a - b)) < 1e-12
+
+
+def test_tilemix_map_rules():
+    T, H, W, band = 300, 40, 40, 2
+    zero = ko.tilemix_map(T, H, W, "zero", 0.5, band).kind
+    one = ko.tilemix_map(T, H, W, "one", 0.5, band).kind
+    assert np.array_equal(ko.tilemix_map(T, H, W, "band", 0.0, band).kind, zero)
+    assert np.array_equal(ko.tilemix_map(T, H, W, "band", 1.0, band).kind, one)
+    nt = zero.shape[0]
+    text = [a * 128 < T for a in range(nt)]
+    for p in (0.25, 0.5, 0.75):
+        kind = ko.tilemix_map(T, H, W, "band", p, band).kind
+        for a in range(nt):
+            n_left = sum(1 for b in range(nt) if not text[a] and not text[b] and abs(a - b) > band)
+            assert (kind[a] & ko.KIND_INT8 > 0).sum() == math.floor(p * n_left + 0.5)
+            for b in range(nt):
+                if text[a] or text[b] or abs(a - b) <= band:
+                    assert not kind[a, b] & ko.KIND_INT8
+        # farthest tiles go first: within a row, every INT8 tile is at least as
+        # far from the diagonal as every FP16 left-over tile
+        for a in range(nt):
+            d8 = [abs(a - b) for b in range(nt) if kind[a, b] & ko.KIND_INT8]
+            d16 = [abs(a - b) for b in range(nt)
+                   if not text[a] and not text[b] and abs(a - b) > band and not kind[a, b] & ko.KIND_INT8]
+            if d8 and d16:
+                assert min(d8) >= max(d16)
+
+
+def test_int8_score_error_bound():
+    c = small_case("tilemix", pattern="one", qk_dist="normal_koffset", head_dim=64, text_len=0,
+                   grid_h=16, grid_w=16, q_heads=2, kv_heads=1)
+    q, k, _, _ = make_inputs(c)
+    qd, kd = f64(q), f64(k)
+    kc, _ = ko.centred_keys(kd)
+    q8, sq = ko.quantize_blocks(qd)
+    k8, sk = ko.quantize_blocks(kc)
+    L = c.seq_len
+    blk = np.arange(L) // 128
+    for h in range(2):
+        Sq = sq[0, h, blk][:, None]
+        Sk = sk[0, 0, blk][None, :]
+        s8 = (q8[0, :, h].astype(np.float64) @ k8[0, :, 0].astype(np.float64).T) * Sq * Sk
+        exact = qd[0, :, h] @ kc[0, :, 0].T
+        bound = (np.abs(qd[0, :, h]).sum(1)[:, None] * Sk / 2 + np.abs(kc[0, :, 0]).sum(1)[None, :] * Sq / 2
+                 + 64 * Sq * Sk / 4)
+        assert np.all(np.abs(s8 - exact) <= bound + 1e-12)
+    # dequantisation error is at most half a step
+    step = sq[0][:, blk].T[:, :, None]                       # [L, Hq, 1]
+    assert np.all(np.abs(q8[0].astype(np.float64) * step - qd[0]) <= step / 2 + 1e-15)
+
+
+def test_quantize_golden_example():
+    g = json.load(open(os.path.join(GOLDEN, "quant_example.json")))
+    x = np.zeros(g["shape"])
+    rows = np.array(g["block0_first_rows"])
+    x[0, :3, 0, :] = rows
+    for prec in ("f64", "f32"):
+        codes, scales = ko.quantize_blocks(x.astype(np.float32) if prec == "f32" else x, prec)
+        assert np.array_equal(codes[0, :3, 0, :], np.array(g["block0_codes"]))
+        assert np.all(codes[0, 3:] == 0)
+        assert float(scales[0, 0, 0]) == g["block0_scale"]
+        assert float(scales[0, 0, 1]) == g["block1_scale"]
+
+
+# --------------------------------------------------------------------------- the pages' numbers
+
+def test_pages_grid_and_window():
+    f = json.load(open(os.path.join(GOLDEN, "pages_facts.json")))
+    side = f["image_px"] // 8 // 2           # VAE latent /8, then halved by the wrapper
+    assert f["image_px"] // 8 == f["latent_side_at_1024"]
+    assert side == f["token_grid_side_at_1024"]
+    assert f["window_default"] // 2 == f["rows_each_side_at_window_11"]
+    assert f["q_heads"] * 128 == f["hidden"]
+    assert abs(128 * 128 + 512 - f["tokens_at_4mp_approx"]) < 1000
+    # an image token in the middle of the 64x64 grid sees exactly rows r-5 .. r+5
+    T, H, W = 16, side, side
+    c, q, k, v = _q_zero_case(mode="scanline", text_len=T, grid_h=H, grid_w=W, window=f["window_default"],
+                              tile_aligned=False, q_heads=1, kv_heads=1, head_dim=64)
+    rows_q = np.array([T + 32 * W + 7])
+    P = ko.attention(c, q, k, v, rows=rows_q, return_probs=True)["probs"][0, 0, 0]
+    seen_rows = sorted({(j - T) // W for j in np.nonzero(P)[0] if j >= T})
+    assert seen_rows == list(range(32 - 5, 32 + 5 + 1))
+    assert np.all(P[:T] > 0)
+
+
+def test_scanline_padding_layout():
+    f = json.load(open(os.path.join(GOLDEN, "pages_facts.json")))
+    phys = ko.logical_layout(300, 64, 64, "scanline")
+    assert ko.text_slot(300) == f["text_pad"]
+    assert phys.shape[0] % 128 == 0
+    assert np.all(phys[:300] == np.arange(300)) and np.all(phys[300:512] == -1)
+    assert phys[512] == 300 and phys[512 + 4095] == 300 + 4095
