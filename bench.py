@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Benchmark of the Krea 2 attention core at the 4 MP shape (dense / band / scanline).
+
+One step = the three attention variants over one batch of synthetic inputs at
+the Krea 2 4 MP shape (512 text tokens + a 128 x 128 token grid, 48 q heads /
+12 kv heads, head_dim 128):
+  * dense: the CFG pair (batch 2), bf16, sigmoid gate, queries in 4096-token slices;
+  * band:  TileMix band, fp16, smooth_k, band +-2 key blocks, 50% of the left-over
+           image-image tiles INT8 (quantiser included);
+  * scanline: bf16, window 11, tile_aligned, text padded to 512.
+FLOPs = 4 * B * Hq * d * (admitted query-key pairs); value = FLOPs / device time.
+
+python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+Under torchrun every rank runs the same step on its own GPU (independent
+problems, no collective on the data path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOP/s at Krea 2 4 MP shape (dense/band/scanline), % of tensor peak"
+WORKLOAD = ("krea2_4mp_attention_step: dense CFG pair B=2 bf16+gate sliced 4096 | TileMix band p=0.5 "
+            "fp16 smooth_k | scanline w11 tile_aligned bf16; 48/12 heads, d=128, 512 text + 128x128 grid")
+TILE = 128
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"bf16": p["bf16_tflops"], "bf16_sustained": p["bf16_tflops_sustained"],
+                "hbm_gbs": p["hbm_gbs"], "source": "measured"}
+    return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- workload
+ONLY_CASE = None  # --case: run one workload alone (for profiling)
+
+
+def step_cases():
+    from synth import inputs as S
+
+    if ONLY_CASE:
+        extra = {c.name: c for c in _step_cases_all()}
+        if ONLY_CASE in extra:
+            return [extra[ONLY_CASE]]
+        return [S.ALL_CASES[ONLY_CASE]()]
+    return _step_cases_all()
+
+
+def _step_cases_all():
+    from synth import inputs as S
+
+    dense = S.cfg_pair_4mp_sliced()
+    band = S.tilemix_band_4mp()
+    scan = S.Case("scanline_4mp", 1, 48, 12, 128, 512, 128, 128, dtype="bf16", mode="scanline", seed=3,
+                  window=11, tile_aligned=True, text_pad=512)
+    return [dense, band, scan]
+
+
+def admitted_pairs(case, K) -> int:
+    """Admitted (query, key) pairs per (batch, q head), from the library's tile map.
+    Dense / TileMix: every pair of real tokens. Scanline with tile_aligned: every
+    pair of real tokens inside an active tile."""
+    L = case.seq_len
+    if case.mode != "scanline":
+        return L * L
+    assert case.tile_aligned
+    rp, col, _ = K.get_map("scanline", case.text_len, case.grid_h, case.grid_w, window=case.window,
+                           tile_aligned=True, text_pad=case.text_pad)
+    T, N = case.text_len, case.grid_h * case.grid_w
+    Pt = case.text_pad or max(512, -(-T // TILE) * TILE)
+
+    def valid_in_tile(t):
+        s0, s1 = t * TILE, t * TILE + TILE
+        return max(0, min(s1, T) - s0) + max(0, min(s1, Pt + N) - max(s0, Pt))
+
+    vt = [valid_in_tile(t) for t in range(len(rp) - 1)]
+    total = 0
+    for a in range(len(rp) - 1):
+        total += vt[a] * sum(vt[b] for b in col[rp[a]:rp[a + 1]])
+    return total
+
+
+def case_flops(case, K) -> float:
+    return 4.0 * case.batch * case.q_heads * case.head_dim * admitted_pairs(case, K)
+
+
+def make_call(case, K, bufs, ws, status):
+    """Closures that launch one variant (all its kernels) on the current stream."""
+    q, k, v, g, out = bufs
+    opts = dict(text_len=case.text_len, grid_h=case.grid_h, grid_w=case.grid_w, mode=case.mode, out=out,
+                pattern=case.pattern, percentage=case.percentage, band_blocks=case.band_blocks,
+                smooth_k=case.smooth_k, window=case.window, tile_aligned=case.tile_aligned,
+                text_pad=case.text_pad, qk_fp32_accumulate=case.qk_fp32_accumulate, status=status)
+    if ws is not None:
+        opts["workspace"] = ws
+    L = case.seq_len
+    if case.q_len:
+        slices = [(s, min(case.q_len, L - s)) for s in range(0, L, case.q_len)]
+    else:
+        slices = [(0, 0)]
+    launches = []
+    for s, n in slices:
+        launches.append(lambda s=s, n=n: K.attention(q, k, v, g, q_start=s, q_len=n, **opts))
+    n_kernels = len(slices) + (4 if case.mode == "tilemix" else 0)  # quantiser: 2 mean + 2 quant kernels
+    return launches, n_kernels
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if "Active" in val and "Not" not in val:
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, device):
+    import diffusion_transformer_attention_bidirectional_b200 as K
+    from synth import inputs as S
+
+    K._lib.lib()
+    cases = step_cases()
+    P = peaks()
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    host, dev_bufs, calls, flops, kernels = [], [], [], [], 0
+    for c in cases:
+        q, k, v, g = S.make_inputs(c)
+        hb = [t.pin_memory() if t is not None else None for t in (q, k, v, g)]
+        db = [t.to(device) if t is not None else None for t in hb]
+        out = torch.empty(q.shape, dtype=torch.float32, device=device)
+        ws = None
+        if c.mode == "tilemix":
+            p = K.make_params(c.batch, c.q_heads, c.kv_heads, c.head_dim, c.text_len, c.grid_h, c.grid_w,
+                              in_dtype=c.dtype, smooth_k=c.smooth_k)
+            ws = torch.empty(K.workspace_bytes("tilemix", c.text_len, c.grid_h, c.grid_w, p), dtype=torch.uint8,
+                             device=device)
+        launches, nk = make_call(c, K, (*db, out), ws, status)
+        host.append((hb, torch.empty(out.shape, dtype=out.dtype, pin_memory=True)))
+        dev_bufs.append((db, out))
+        calls.append(launches)
+        flops.append(case_flops(c, K))
+        kernels += nk
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)  # 256 MB > 126 MB L2
+
+    def step(timed_events=None):
+        for vi, launches in enumerate(calls):
+            for li, fn in enumerate(launches):
+                if timed_events is not None:
+                    timed_events[vi][li][0].record(stream)
+                fn()
+                if timed_events is not None:
+                    timed_events[vi][li][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during warm-up")
+
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    sampler.start()
+    per_step = []
+    var_ms = [0.0] * len(calls)
+    attn_dense_ms = 0.0
+    for _ in range(args.steps):
+        flush.zero_()  # evict L2 between steps, outside the timed span
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in l]
+              for l in calls]
+        step(ev)
+        torch.cuda.synchronize(device)
+        tot = 0.0
+        for vi, l in enumerate(ev):
+            ms = ev[vi][0][0].elapsed_time(ev[vi][-1][1])
+            var_ms[vi] += ms
+            tot += ms
+            if vi == 0:
+                attn_dense_ms += sum(a.elapsed_time(b) for a, b in l)
+        per_step.append(tot)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during timing")
+    step_ms = sum(per_step) / len(per_step)
+    if world > 1:
+        t = torch.tensor([step_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_ms = float(t.item())
+    total_flops = sum(flops)
+    value = world * total_flops / (step_ms * 1e-3) / 1e12
+
+    # e2e through the public API with host buffers: pinned H2D of every input,
+    # the step, D2H of every output, all inside the timed span
+    e2e_steps = max(1, min(args.steps, 3))
+    h2d = sum(t.numel() * t.element_size() for hb, _ in host for t in hb if t is not None)
+    d2h = sum(o.numel() * o.element_size() for _, o in host)
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for (hb, hout), (db, dout) in zip(host, dev_bufs):
+            for h_, d_ in zip(hb, db):
+                if h_ is not None:
+                    d_.copy_(h_, non_blocking=True)
+        step()
+        for (hb, hout), (db, dout) in zip(host, dev_bufs):
+            hout.copy_(dout, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * total_flops / (e2e_ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel: the attention kernel on the dense variant
+    # (its launches are attention kernels only), algorithmic FLOPs / event time
+    dense_attn_ms = attn_dense_ms / args.steps
+    achieved = flops[0] / (dense_attn_ms * 1e-3) / 1e12
+    names = [c.name for c in cases]
+    variants = {}
+    for i, c in enumerate(cases):
+        ms = var_ms[i] / args.steps
+        tf = flops[i] / (ms * 1e-3) / 1e12
+        pk = P["bf16"]
+        if c.mode == "tilemix":
+            # blended peak: INT8 halves only the QK^T half of INT8 tiles; INT8 peak taken
+            # as 2x the measured bf16 peak (the datasheet ratio 4.5 / 2.25 PFLOP/s)
+            rp, col, kind = K.get_map("tilemix", c.text_len, c.grid_h, c.grid_w, pattern=c.pattern,
+                                      percentage=c.percentage, band_blocks=c.band_blocks)
+            n8 = int(((kind & 2) > 0).sum())
+            f8 = flops[i] * (n8 / len(kind)) / 2
+            pk = flops[i] / ((flops[i] - f8) / P["bf16"] + f8 / (2 * P["bf16"]))
+        variants[names[i]] = {"ms": round(ms, 4), "tflops": round(tf, 1), "peak_tflops": round(pk, 1),
+                              "frac_of_peak": round(tf / pk, 4), "gflop": round(flops[i] / 1e9, 1)}
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": world * 4, "seq_len": cases[0].seq_len,
+                   "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MB write)"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": P["bf16"], "unit": "TFLOP/s",
+                     "frac": round(achieved / P["bf16"], 4), "traffic": None,
+                     "kernel": "attn_fwd_kernel<bf16> (dense CFG pair, 5 slices)",
+                     "peak_source": f"{P['source']} bf16 burst"},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": kernels * args.steps,
+        "variants": variants,
+    }
+    if clocks:
+        res["clocks"] = clocks
+    return res
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+def oracle_sample(rows_per_variant: int):
+    """Time the fp64 oracle on a bounded sample of the same workload: the first
+    `rows_per_variant` query rows of every variant, all heads, batch 0."""
+    from oracle import krea_oracle as ko
+    from synth import inputs as S
+
+    import diffusion_transformer_attention_bidirectional_b200 as K
+
+    cases = step_cases()
+    data = [S.make_inputs(c) for c in cases]
+    t_total, f_total = 0.0, 0.0
+    for c, (q, k, v, g) in zip(cases, data):
+        rows = np.arange(rows_per_variant)
+        L = c.seq_len
+        if c.mode == "scanline":
+            frac = admitted_pairs(c, K) / (L * L)  # average admitted share per row
+        else:
+            frac = 1.0
+        t0 = time.perf_counter()
+        ko.attention(c, q, k, v, g, rows=rows, batches=[0])
+        t_total += time.perf_counter() - t0
+        f_total += 4.0 * c.q_heads * c.head_dim * rows_per_variant * L * frac
+    return f_total, t_total
+
+
+def cpu_cores():
+    try:
+        import threadpoolctl
+
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"), default=None)
+        if n:
+            return n
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args):
+    rows = 32
+    oracle_sample(8)  # untimed warm-up of numpy / BLAS
+    times = []
+    for _ in range(args.warmup):
+        oracle_sample(rows)
+    for _ in range(args.steps):
+        f, t = oracle_sample(rows)
+        times.append((f, t))
+    f = sum(x[0] for x in times)
+    t = sum(x[1] for x in times)
+    value = f / t / 1e12
+    sample = f"first {rows} query rows of each variant, all 48 heads, batch 0 (fp64 numpy oracle)"
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None,
+                    help="profile one workload alone (a synth.inputs case or a step variant name)")
+    args = ap.parse_args()
+    global ONLY_CASE
+    ONLY_CASE = args.case
+    if args.case:
+        args.no_cpu_baseline = True
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    try:
+        res = run_ours(args, rank, world, device)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            rows = 64
+            f, t = oracle_sample(rows)
+            res["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
+                                   "kind": "oracle",
+                                   "sample": f"first {rows} query rows of each variant, all 48 heads, batch 0; "
+                                             f"{t:.1f} s of fp64 numpy"}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

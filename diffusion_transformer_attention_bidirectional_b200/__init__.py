@@ -1,0 +1,182 @@
+"""Krea 2 bidirectional DiT attention core on B200 (sm_100a).
+
+Python binding of libkrea_attn.so (C ABI in include/krea_attn.h). This module
+only marshals arguments -- tensor pointers, strides, dtypes and the CUDA stream
+-- and allocates outputs and workspace through torch; every step of the
+attention runs in the library's CUDA kernels. There is no CPU path: calls on
+tensors that are not on a CUDA device are rejected.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import KreaError, Params, check, lib
+
+__all__ = ["attention", "quantize", "get_map", "map_size", "workspace_bytes", "workspace_layout",
+           "make_params", "clear_cache", "KreaError"]
+
+_TORCH_DT = {torch.float16: "f16", torch.bfloat16: "bf16", torch.float32: "f32"}
+
+
+def make_params(batch: int, q_heads: int, kv_heads: int, head_dim: int, text_len: int, grid_h: int,
+                grid_w: int, *, in_dtype: str = "bf16", out_dtype: str = "f32", softmax_scale: float = 0.0,
+                q_start: int = 0, q_len: int = 0, pattern: str = "band", percentage: float = 0.5,
+                band_blocks: int = 2, smooth_k: bool = True, qk_fp32_accumulate: bool = False,
+                window: int = 11, tile_aligned: bool = True, text_pad: int = 0,
+                debug_wait_limit: int = 0, debug_flags: int = 0) -> Params:
+    """krea_attn_params_t for contiguous [B, L, H, d] tensors (strides fixed up by `attention`)."""
+    p = Params()
+    lib().krea_attn_default_params(ctypes.byref(p), batch, q_heads, kv_heads, head_dim, text_len, grid_h,
+                                   grid_w)
+    p.in_dtype = _lib.DTYPE[in_dtype]
+    p.out_dtype = _lib.DTYPE[out_dtype]
+    p.softmax_scale = float(softmax_scale)
+    p.q_start = int(q_start)
+    p.q_len = int(q_len)
+    p.pattern = _lib.PATTERN[pattern]
+    p.percentage = float(percentage)
+    p.band_blocks = int(band_blocks)
+    p.smooth_k = int(bool(smooth_k))
+    p.qk_fp32_accumulate = int(bool(qk_fp32_accumulate))
+    p.window = int(window)
+    p.tile_aligned = int(bool(tile_aligned))
+    p.text_pad = int(text_pad)
+    p.debug_wait_limit = int(debug_wait_limit)
+    p.debug_flags = int(debug_flags)
+    return p
+
+
+def _set_strides(arr, t: torch.Tensor) -> None:
+    s = t.stride()
+    if t.dim() != 4 or s[3] != 1:
+        raise ValueError("expected a [batch, tokens, heads, head_dim] tensor with head_dim contiguous")
+    arr[0], arr[1], arr[2] = s[0], s[1], s[2]
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream], device: torch.device) -> int:
+    st = stream if stream is not None else torch.cuda.current_stream(device)
+    return int(st.cuda_stream)
+
+
+def workspace_bytes(mode: str, text_len: int, grid_h: int, grid_w: int, params: Params) -> int:
+    return int(lib().krea_attn_workspace_bytes(text_len, grid_h, grid_w, _lib.MODE[mode], ctypes.byref(params)))
+
+
+def workspace_layout(text_len: int, grid_h: int, grid_w: int, params: Params) -> dict:
+    w = _lib.WsLayout()
+    check(lib().krea_attn_workspace_layout(text_len, grid_h, grid_w, _lib.MODE["tilemix"], ctypes.byref(params),
+                                           ctypes.byref(w)), "workspace_layout")
+    return {n: int(getattr(w, n)) for n, _ in w._fields_}
+
+
+def map_size(mode: str, text_len: int, grid_h: int, grid_w: int, params: Params):
+    nt, nnz = ctypes.c_int32(), ctypes.c_int32()
+    check(lib().krea_attn_map_size(text_len, grid_h, grid_w, _lib.MODE[mode], ctypes.byref(params),
+                                   ctypes.byref(nt), ctypes.byref(nnz)), "map_size")
+    return nt.value, nnz.value
+
+
+def get_map(mode: str, text_len: int, grid_h: int, grid_w: int, params: Optional[Params] = None, **opts):
+    """Host copy of the tile map: (row_ptr[n_tiles+1], col[nnz], kind[nnz]) as numpy arrays."""
+    if params is None:
+        params = make_params(1, 1, 1, 128, text_len, grid_h, grid_w, **opts)
+    nt, nnz = map_size(mode, text_len, grid_h, grid_w, params)
+    row_ptr = np.zeros(nt + 1, dtype=np.int32)
+    col = np.zeros(max(nnz, 1), dtype=np.int32)
+    kind = np.zeros(max(nnz, 1), dtype=np.uint8)
+    check(lib().krea_attn_get_map(text_len, grid_h, grid_w, _lib.MODE[mode], ctypes.byref(params),
+                                  row_ptr.ctypes.data, col.ctypes.data, kind.ctypes.data, nnz), "get_map")
+    return row_ptr, col[:nnz], kind[:nnz]
+
+
+def _check_inputs(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("krea attention runs on CUDA tensors only")
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[torch.Tensor] = None, *,
+              text_len: int, grid_h: int, grid_w: int, mode: str = "dense",
+              out: Optional[torch.Tensor] = None, out_dtype: Optional[torch.dtype] = torch.float32,
+              workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None, **opts) -> torch.Tensor:
+    """out = sigmoid(gate) * softmax(scale q k^T over the admitted keys) v, per query head.
+
+    q [B, L, Hq, d], k and v [B, L, Hkv, d], gate [B, L, Hq, d] or None; L = text_len + grid_h * grid_w.
+    mode: "dense" | "tilemix" | "scanline"; `opts` are make_params keywords (q_start, q_len,
+    pattern, percentage, band_blocks, smooth_k, window, tile_aligned, text_pad, ...).
+    """
+    _check_inputs(q, k, v, gate, out, workspace, status)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    in_dt = _TORCH_DT[q.dtype]
+    if out is None:
+        odt = out_dtype if out_dtype is not None else q.dtype
+        out = torch.empty((B, L, Hq, d), dtype=odt, device=q.device)
+    p = make_params(B, Hq, Hkv, d, text_len, grid_h, grid_w, in_dtype=in_dt, out_dtype=_TORCH_DT[out.dtype],
+                    **opts)
+    _set_strides(p.q_stride, q)
+    _set_strides(p.k_stride, k)
+    _set_strides(p.v_stride, v)
+    _set_strides(p.out_stride, out)
+    if gate is not None:
+        _set_strides(p.gate_stride, gate)
+    if mode == "tilemix":
+        need = workspace_bytes(mode, text_len, grid_h, grid_w, p)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        p.workspace = workspace.data_ptr()
+        p.workspace_bytes = workspace.numel() * workspace.element_size()
+    if status is not None:
+        p.status = status.data_ptr()
+    rc = lib().krea_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                             gate.data_ptr() if gate is not None else None, out.data_ptr(),
+                             text_len, grid_h, grid_w, _lib.MODE[mode], ctypes.byref(p),
+                             _stream_ptr(stream, q.device))
+    check(rc, "krea_attn_fwd")
+    return out
+
+
+def quantize(q: torch.Tensor, k: torch.Tensor, *, text_len: int, grid_h: int, grid_w: int,
+             smooth_k: bool = True, workspace: Optional[torch.Tensor] = None,
+             stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Run only the TileMix quantiser; returns views of the workspace:
+    kc (centred keys), q8, k8, sq, sk, mu."""
+    _check_inputs(q, k, workspace)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    p = make_params(B, Hq, Hkv, d, text_len, grid_h, grid_w, in_dtype=_TORCH_DT[q.dtype], smooth_k=smooth_k)
+    _set_strides(p.q_stride, q)
+    _set_strides(p.k_stride, k)
+    lay = workspace_layout(text_len, grid_h, grid_w, p)
+    if workspace is None:
+        workspace = torch.empty(lay["total"], dtype=torch.uint8, device=q.device)
+    p.workspace = workspace.data_ptr()
+    p.workspace_bytes = workspace.numel()
+    check(lib().krea_attn_quantize(q.data_ptr(), k.data_ptr(), text_len, grid_h, grid_w, ctypes.byref(p),
+                                   _stream_ptr(stream, q.device)), "krea_attn_quantize")
+    nt = (L + _lib.TILE - 1) // _lib.TILE
+
+    def view(off, n, dt, shape):
+        return workspace[off:off + n * torch.tensor([], dtype=dt).element_size()].view(dt).view(shape)
+
+    res = {
+        "q8": view(lay["q8"], B * L * Hq * d, torch.int8, (B, L, Hq, d)),
+        "k8": view(lay["k8"], B * L * Hkv * d, torch.int8, (B, L, Hkv, d)),
+        "sq": view(lay["sq"], B * Hq * nt, torch.float32, (B, Hq, nt)),
+        "sk": view(lay["sk"], B * Hkv * nt, torch.float32, (B, Hkv, nt)),
+        "workspace": workspace,
+    }
+    if smooth_k:
+        res["kc"] = view(lay["kc"], B * L * Hkv * d, q.dtype, (B, L, Hkv, d))
+        res["mu"] = view(lay["mu"], B * Hkv * d, torch.float32, (B, Hkv, d))
+    return res
+
+
+def clear_cache() -> None:
+    lib().krea_attn_clear_cache()

@@ -1,0 +1,606 @@
+// Attention kernel of the Krea 2 core for B200 (sm_100a): bidirectional
+// online-softmax attention over 128 x 128 score tiles listed by a tile map,
+// FP16/BF16 or INT8 QK^T on tcgen05 tensor cores with TMEM accumulators,
+// K/V tiles staged by TMA, sigmoid(gate) fused into the epilogue.
+//
+// What it computes ("Krea 2 TileMix Attention (FP16/INT8 tiles)", section "What
+// it actually patches"; "Krea 2 Scanline Attention", section "What the mask
+// actually is"; "LayerStream: Krea2 Chunking", section "What the node does to
+// the block"):
+//   out[b,t,h,:] = sigmoid(gate[b,t,h,:]) * sum_j softmax_j(scale * s(t,j)) v[b,j,h/rep,:]
+// over the key tiles of the query tile's map row, in ascending key-tile order;
+// masked tiles apply the padding / scanline predicate per key slot, skipped
+// tiles are never loaded.
+//
+// One CTA = one 128-row query tile of TWO query heads that share a kv head
+// (GQA resolved by index: kv head = h / rep), so every K/V tile loaded from HBM
+// feeds two 128 x 128 x d products. Warp roles (384 threads, 3 warpgroups):
+//   warps 0-3  softmax for head 0 (thread = query row), epilogue
+//   warps 4-7  softmax for head 1
+//   warp  8    TMA producer: Q once, then K_j, V_j into a 4-slot ring of 32 KB
+//   warp  9    TMEM allocator and the single thread issuing tcgen05.mma
+//   warps 10-11 idle (they complete the third warpgroup)
+// The launch gives 168 registers per thread; the producer/MMA warpgroup drops to
+// 56 (setmaxnreg.dec) so the two softmax warpgroups can rise to 224 and keep a
+// whole 128-score row in registers: 32*56 + 2*32*224 = 3*32*168 per SM
+// sub-partition. The host refuses to launch unless the kernel was compiled to
+// exactly 168 registers, so the raise can never wait for registers that are
+// not there.
+// TMEM (512 columns x 128 lanes): S0 [0,128) S1 [128,256) O0 [256,384)
+// O1 [384,512); P_i (16-bit, 64 columns) overwrites the first half of S_i.
+// Per kv tile j and head i the MMA thread issues, in order,
+//   PV_i(j-1): O_i += P_i V_{j-1}   then   QK_i(j): S_i = Q_i K_j^T
+// and commits S_i after QK_i(j); tcgen05 operations of one thread complete in
+// issue order, so when softmax i sees S_i(j) complete, PV_i(j-1) is complete
+// too and O_i may be rescaled in place before P_i(j) is released.
+// The running max is only moved when it grows by more than 2^8 (lazy rescale):
+// exact, since numerator and denominator share the stale maximum.
+//
+// Every barrier wait is bounded (p.wait_limit SM cycles): a wait that runs out
+// sets a CTA abort flag and writes KREA_ERR_DEVICE_TIMEOUT to p.status; the
+// producer then waits (bounded) for its own TMA copies in flight, the MMA thread
+// for its own MMAs, and the CTA frees its TMEM and exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "krea_internal.h"
+#include "ptx_sm100.cuh"
+
+namespace krea {
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kOtherRegs = 56;
+constexpr int kSlots = 4;
+constexpr uint32_t kBox = 16384;       // one TMA box: 128 rows x 128 bytes
+constexpr uint32_t kTileBytes = 32768; // 128 x 128 16-bit
+constexpr uint32_t SM_Q = 0;           // 2 x 32 KB
+constexpr uint32_t SM_Q8 = 65536;      // 2 x 16 KB
+constexpr uint32_t SM_SLOT = 98304;    // kSlots x 32 KB
+constexpr uint32_t SM_BAR = SM_SLOT + kSlots * kTileBytes;
+constexpr int BAR_Q = 0, BAR_FULL = 1, BAR_EMPTY = BAR_FULL + kSlots, BAR_S = BAR_EMPTY + kSlots,
+              BAR_P = BAR_S + 2, BAR_O = BAR_P + 2, BAR_DRAIN = BAR_O + 2, BAR_NEVER = BAR_DRAIN + 1,
+              N_BARS = BAR_NEVER + 1;
+constexpr uint32_t SM_TMEM_PTR = SM_BAR + 8 * N_BARS;
+constexpr uint32_t SM_ABORT = SM_TMEM_PTR + 4;
+constexpr uint32_t SMEM_USED = SM_BAR + 256;
+constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // slack to align the base to 1024 bytes
+static_assert(8 * N_BARS + 8 <= 256, "barrier block overflow");
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+constexpr long long kDrainLimit = 4000000000LL;
+constexpr float kNegInf = -INFINITY;
+
+struct Ctl {
+  volatile int* abort;
+  int32_t* status;
+  long long limit;
+};
+
+__device__ __forceinline__ void raise_timeout(const Ctl& c) {
+  *c.abort = 1;
+  if (c.status) atomicCAS(c.status, 0, KREA_ERR_DEVICE_TIMEOUT);
+}
+
+// Single-thread bounded wait.
+__device__ __forceinline__ bool wait1(const Ctl& c, uint32_t bar, uint32_t parity) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*c.abort) return false;
+    if (clock64() - t0 > c.limit) {
+      raise_timeout(c);
+      return false;
+    }
+  }
+}
+
+// Whole-warp bounded wait: every lane polls, the warp leaves together.
+__device__ __forceinline__ bool wait_warp(const Ctl& c, uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (true) {
+    const bool done = ptx::mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    const bool stop = *c.abort || (clock64() - t0 > c.limit);
+    if (__any_sync(0xffffffffu, stop)) {
+      if ((threadIdx.x & 31) == 0 && !*c.abort) raise_timeout(c);
+      return false;
+    }
+  }
+}
+
+// Wait used only on the abort path, for work this thread itself started.
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!ptx::mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kDrainLimit) return;
+}
+
+// First physical token of logical tile `tile` (text slots map to themselves,
+// image slots start at Pt).
+__device__ __forceinline__ int tile_row0(int tile, const AttnDevParams& p) {
+  const int s0 = tile * kTile;
+  return s0 < p.Pt ? s0 : s0 - p.Pt + p.T;
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (BF16) return ptx::pack_bf16(lo, hi);
+  else return ptx::pack_f16(lo, hi);
+}
+
+template <bool BF16>
+__device__ __forceinline__ float h2f(uint16_t u) {
+  if constexpr (BF16) return __uint_as_float((uint32_t)u << 16);
+  else {
+    float f;
+    asm("{\n\t.reg .f16 t;\n\tmov.b16 t, %1;\n\tcvt.f32.f16 %0, t;\n\t}" : "=f"(f) : "h"(u));
+    return f;
+  }
+}
+
+__device__ __forceinline__ float sigmoidf_(float x) { return __frcp_rn(1.0f + __expf(-x)); }
+
+// 2^x on the FMA pipe for a pair of values, so that part of the exponentials
+// leaves the MUFU unit (whose 16 results per clock per SM would otherwise bound
+// the softmax). Range reduction x = n + f with n = rint(x), f in [-1/2, 1/2]
+// (rounding by adding 1.5 * 2^23), a polynomial for 2^f, and 2^n applied by
+// adding n to the exponent field. The polynomial keeps p(0) = 1 exactly and is a
+// minimax fit of the relative error of 2^f on [-1/2, 1/2] (Lawson's iteratively
+// reweighted least squares): degree 3, max relative error 1.2e-4, for bf16
+// probabilities (8-bit significand); degree 4, 2.9e-6, for fp16 (11-bit).
+// x is clamped to -127, where the result is exactly 0 (masked keys stay 0).
+template <bool BF16>
+__device__ __forceinline__ void exp2_poly2(float& a, float& b) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  a = fmaxf(a, -127.0f);
+  b = fmaxf(b, -127.0f);
+  const uint64_t x = ptx::f2(a, b);
+  const uint64_t j = ptx::add2(x, ptx::f2(kRound, kRound));
+  const uint64_t n = ptx::add2(j, ptx::f2(-kRound, -kRound));
+  float n0, n1;
+  ptx::unf2(n, n0, n1);
+  const uint64_t f = ptx::add2(x, ptx::f2(-n0, -n1));
+  uint64_t p;
+  if constexpr (BF16) {
+    p = ptx::fma2(ptx::f2(0.055417872965335846f, 0.055417872965335846f), f,
+                  ptx::f2(0.242211252450943f, 0.242211252450943f));
+    p = ptx::fma2(p, f, ptx::f2(0.6931995153427124f, 0.6931995153427124f));
+  } else {
+    p = ptx::fma2(ptx::f2(0.009585633873939514f, 0.009585633873939514f), f,
+                  ptx::f2(0.05590590462088585f, 0.05590590462088585f));
+    p = ptx::fma2(p, f, ptx::f2(0.2402404099702835f, 0.2402404099702835f));
+    p = ptx::fma2(p, f, ptx::f2(0.6931242942810059f, 0.6931242942810059f));
+  }
+  p = ptx::fma2(p, f, ptx::f2(1.0f, 1.0f));
+  float p0, p1, j0, j1;
+  ptx::unf2(p, p0, p1);
+  ptx::unf2(j, j0, j1);
+  // the low mantissa bits of j hold n; shifting them into the exponent field
+  a = __int_as_float(__float_as_int(p0) + (__float_as_int(j0) << 23));
+  b = __int_as_float(__float_as_int(p1) + (__float_as_int(j1) << 23));
+}
+
+// Exact int32 -> fp32 for |x| < 2^22 on the integer and FMA pipes (the INT8
+// tile sums are bounded by 128 * 127 * 127 < 2^21).
+__device__ __forceinline__ float i2f_exact(uint32_t x) {
+  return __int_as_float((int)(x + 0x4B400000u)) - 12582912.0f;
+}
+
+// Online-softmax step of one 128-key tile for one query row held by this thread.
+// v: the row of S (fp32 bits, or s32 for INT8 tiles), overwritten. mult: score
+// scale in log2 units (softmax scale * log2 e, times s_q s_k for INT8 tiles).
+// Key column c is admitted iff c < a1 or a2 <= c < a3 (masked tiles only).
+// Writes P (16-bit pairs) over the first 64 columns of S; updates m, l and,
+// when the running maximum moves, rescales O in TMEM.
+template <bool BF16, bool IS8, bool MASKED, bool ALL_POLY>
+__device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int a1, int a2, int a3, float& m,
+                                             float& l, bool first, uint32_t tS, uint32_t tO, int d) {
+#pragma unroll
+  for (int c = 0; c < 128; ++c) {
+    float r = IS8 ? i2f_exact(v[c]) : __uint_as_float(v[c]);
+    if constexpr (MASKED) r = ((c < a1) || (c >= a2 && c < a3)) ? r : kNegInf;
+    v[c] = __float_as_uint(r);
+  }
+  float mx0 = kNegInf, mx1 = kNegInf;
+#pragma unroll
+  for (int c = 0; c < 128; c += 4) {
+    mx0 = ptx::max3(mx0, __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+    mx1 = ptx::max3(mx1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+  }
+  const float m_tile = fmaxf(mx0, mx1) * mult;  // mult > 0
+  const float m_new = fmaxf(m, m_tile);
+  if (first) {
+    m = m_new;
+  } else {
+    const bool need = m_new > m + 8.0f;
+    if (__any_sync(0xffffffffu, need)) {
+      const float f = need ? ptx::ex2(m - m_new) : 1.0f;
+      for (int j = 0; j < d / 32; ++j) {
+        uint32_t o[32];
+        __syncwarp();
+        ptx::tmem_ld32(tO + 32u * j, o);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+        ptx::tmem_st32(tO + 32u * j, o);
+      }
+      if (need) {
+        l *= f;
+        m = m_new;
+      }
+    }
+  }
+  const float m_use = (m == kNegInf) ? 0.f : m;
+  const uint64_t mult2 = ptx::f2(mult, mult), negm2 = ptx::f2(-m_use, -m_use);
+  uint64_t acc0 = ptx::f2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {  // 64 keys -> 32 columns of P per half
+    uint32_t pk[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int c = 64 * h + 2 * i;
+      const uint64_t x = ptx::fma2(ptx::f2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), mult2, negm2);
+      float p0, p1;
+      ptx::unf2(x, p0, p1);
+      if (ALL_POLY || (i & 3) == 3) {
+        exp2_poly2<BF16>(p0, p1);
+      } else {
+        p0 = ptx::ex2(p0);
+        p1 = ptx::ex2(p1);
+      }
+      if (i & 1) acc1 = ptx::add2(acc1, ptx::f2(p0, p1));
+      else acc0 = ptx::add2(acc0, ptx::f2(p0, p1));
+      pk[i] = pack2<BF16>(p0, p1);
+    }
+    ptx::tmem_st32(tS + 32u * h, pk);
+  }
+  float s0, s1, s2, s3;
+  ptx::unf2(acc0, s0, s1);
+  ptx::unf2(acc1, s2, s3);
+  l += (s0 + s1) + (s2 + s3);
+}
+
+// ---------------------------------------------------------------------------
+template <bool BF16, bool ALL_POLY>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q8,
+                    const __grid_constant__ CUtensorMap tm_k8, const __grid_constant__ AttnDevParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sb = smem_raw + (base - raw);
+
+  // work item: (batch, kv head, head pair, query tile), query tile fastest
+  int idx = blockIdx.x;
+  const int qt = p.tile_begin + idx % p.n_slice_tiles;
+  idx /= p.n_slice_tiles;
+  const int pair = idx % p.npairs;
+  idx /= p.npairs;
+  const int g = idx % p.Hkv;
+  const int b = idx / p.Hkv;
+  const int h0 = g * p.rep + pair * p.nh;
+  const int e0 = p.row_ptr[qt];
+  const int n = p.row_ptr[qt + 1] - e0;
+  if (n <= 0) return;  // a tile of padding slots only
+  // fail fast: once any CTA of this launch (or an earlier one) has given up, do no work
+  if (p.status && *reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto bar = [&](int i) { return base + SM_BAR + 8u * (uint32_t)i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sb + SM_ABORT);
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sb + SM_TMEM_PTR);
+  const Ctl ctl{abort_flag, p.status, p.wait_limit};
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar(BAR_Q), 1);
+    for (int i = 0; i < kSlots; ++i) {
+      ptx::mbar_init(bar(BAR_FULL + i), 1);
+      ptx::mbar_init(bar(BAR_EMPTY + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(bar(BAR_S + i), 1);
+      ptx::mbar_init(bar(BAR_P + i), 4);  // one arrival per softmax warp
+      ptx::mbar_init(bar(BAR_O + i), 1);
+    }
+    ptx::mbar_init(bar(BAR_DRAIN), 1);
+    ptx::mbar_init(bar(BAR_NEVER), 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_ptr), 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+  const int nh = p.nh;
+  const int d = p.d;
+
+  if (warp >= 8) {
+  ptx::regs_dec<kOtherRegs>();  // the whole third warpgroup
+  if (warp == 8) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tm_q);
+      ptx::prefetch_tmap(&tm_k);
+      ptx::prefetch_tmap(&tm_v);
+      bool has_int8 = false;
+      for (int t = 0; t < n; ++t) has_int8 |= (p.entries[e0 + t] & KREA_KIND_INT8) != 0;
+      const int nbox = d / 64;
+      const int qrow0 = tile_row0(qt, p);
+      ptx::mbar_arrive_expect_tx(bar(BAR_Q), nh * nbox * kBox + (has_int8 ? nh * kBox : 0));
+      for (int i = 0; i < nh; ++i) {
+        for (int x = 0; x < nbox; ++x)
+          ptx::tma_load_4d(base + SM_Q + i * kTileBytes + x * kBox, &tm_q, bar(BAR_Q), x * 64, h0 + i, qrow0, b);
+        if (has_int8) ptx::tma_load_4d(base + SM_Q8 + i * kBox, &tm_q8, bar(BAR_Q), 0, h0 + i, qrow0, b);
+      }
+      uint32_t it = 0;
+      for (int t = 0; t < n; ++t) {
+        const int e = p.entries[e0 + t];
+        const int krow0 = tile_row0(e >> 2, p);
+        // K tile (INT8 codes for INT8 tiles)
+        uint32_t slot = it % kSlots;
+        if (!wait1(ctl, bar(BAR_EMPTY + slot), ((it / kSlots) & 1) ^ 1)) break;
+        uint32_t dst = base + SM_SLOT + slot * kTileBytes;
+        if (e & KREA_KIND_INT8) {
+          ptx::mbar_arrive_expect_tx(bar(BAR_FULL + slot), kBox);
+          ptx::tma_load_4d(dst, &tm_k8, bar(BAR_FULL + slot), 0, g, krow0, b);
+        } else {
+          ptx::mbar_arrive_expect_tx(bar(BAR_FULL + slot), nbox * kBox);
+          for (int x = 0; x < nbox; ++x)
+            ptx::tma_load_4d(dst + x * kBox, &tm_k, bar(BAR_FULL + slot), x * 64, g, krow0, b);
+        }
+        ++it;
+        // V tile
+        slot = it % kSlots;
+        if (!wait1(ctl, bar(BAR_EMPTY + slot), ((it / kSlots) & 1) ^ 1)) break;
+        dst = base + SM_SLOT + slot * kTileBytes;
+        ptx::mbar_arrive_expect_tx(bar(BAR_FULL + slot), nbox * kBox);
+        for (int x = 0; x < nbox; ++x)
+          ptx::tma_load_4d(dst + x * kBox, &tm_v, bar(BAR_FULL + slot), x * 64, g, krow0, b);
+        ++it;
+      }
+      // Every copy this thread started lands before the CTA may exit (already
+      // true on the normal path, where the MMA thread consumed them all).
+      wait_drain(bar(BAR_Q), 0);
+      for (uint32_t j = (it > kSlots ? it - kSlots : 0); j < it; ++j)
+        wait_drain(bar(BAR_FULL + j % kSlots), (j / kSlots) & 1);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t ab = BF16 ? 1u : 0u;
+      const uint32_t id_qk = ptx::idesc(1, ab, 0, 0, 128, 128);
+      const uint32_t id_qk8 = ptx::idesc(2, 1, 0, 0, 128, 128);
+      const uint32_t id_pv = ptx::idesc(1, ab, 0, 1, (uint32_t)d, 128);
+      const int ksteps = d / 16;
+      auto issue_qk = [&](int i, int kind, uint32_t slot) {
+        const uint32_t dS = tmem + (uint32_t)i * 128u;
+        const uint32_t kaddr = base + SM_SLOT + slot * kTileBytes;
+        if (kind & KREA_KIND_INT8) {
+          const uint32_t qaddr = base + SM_Q8 + (uint32_t)i * kBox;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)  // K = 32 bytes per step
+            ptx::mma_i8_ss(dS, ptx::sdesc(qaddr + 32 * k, 16, 1024), ptx::sdesc(kaddr + 32 * k, 16, 1024),
+                           id_qk8, k > 0);
+        } else {
+          const uint32_t qaddr = base + SM_Q + (uint32_t)i * kTileBytes;
+          for (int k = 0; k < ksteps; ++k) {  // K = 16 elements (32 bytes) per step
+            const uint32_t off = (uint32_t)(k >> 2) * kBox + (uint32_t)(k & 3) * 32;
+            ptx::mma_f16_ss(dS, ptx::sdesc(qaddr + off, 16, 1024), ptx::sdesc(kaddr + off, 16, 1024), id_qk,
+                            k > 0);
+          }
+        }
+      };
+      auto issue_pv = [&](int i, uint32_t slot, bool acc) {
+        const uint32_t dO = tmem + 256u + (uint32_t)i * 128u;
+        const uint32_t aP = tmem + (uint32_t)i * 128u;
+        const uint32_t vaddr = base + SM_SLOT + slot * kTileBytes;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // 16 keys per step: 8 TMEM columns of P, 16 V rows
+          ptx::mma_f16_ts(dO, aP + 8u * k, ptx::sdesc(vaddr + 2048u * k, kBox, 1024), id_pv, (acc || k > 0));
+      };
+      bool ok = wait1(ctl, bar(BAR_Q), 0);
+      uint32_t it = 0;
+      if (ok) {
+        ptx::tc_fence_after();
+        ok = wait1(ctl, bar(BAR_FULL + 0), 0);
+      }
+      if (ok) {
+        ptx::tc_fence_after();
+        const int kind0 = p.entries[e0] & 3;
+        for (int i = 0; i < nh; ++i) {
+          issue_qk(i, kind0, 0);
+          ptx::tc_commit(bar(BAR_S + i));
+        }
+        ptx::tc_commit(bar(BAR_EMPTY + 0));
+        it = 1;
+        for (int t = 0; t < n && ok; ++t) {
+          const uint32_t slot_v = it % kSlots;
+          ok = wait1(ctl, bar(BAR_FULL + slot_v), (it / kSlots) & 1);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          ++it;
+          const bool has_next = t + 1 < n;
+          const uint32_t slot_k = it % kSlots;
+          const int kind_next = has_next ? (p.entries[e0 + t + 1] & 3) : 0;
+          for (int i = 0; i < nh && ok; ++i) {
+            ok = wait1(ctl, bar(BAR_P + i), t & 1);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_pv(i, slot_v, t > 0);
+            if (has_next) {
+              if (i == 0) {
+                ok = wait1(ctl, bar(BAR_FULL + slot_k), (it / kSlots) & 1);
+                if (!ok) break;
+                ptx::tc_fence_after();
+              }
+              issue_qk(i, kind_next, slot_k);
+              ptx::tc_commit(bar(BAR_S + i));
+            }
+          }
+          if (!ok) break;
+          ptx::tc_commit(bar(BAR_EMPTY + slot_v));
+          if (has_next) {
+            ptx::tc_commit(bar(BAR_EMPTY + slot_k));
+            ++it;
+          }
+        }
+      }
+      if (ok)
+        for (int i = 0; i < nh; ++i) ptx::tc_commit(bar(BAR_O + i));
+      // every MMA this thread issued finishes before TMEM is freed, also when a
+      // softmax warp gave up waiting on O
+      ptx::tc_commit(bar(BAR_DRAIN));
+      wait_drain(bar(BAR_DRAIN), 0);
+    }
+  }
+  } else {
+    // ------------------------------------------------------------- softmax
+    ptx::regs_inc<kSoftmaxRegs>();
+    const int wg = warp >> 2, wq = warp & 3;
+    if (wg < nh) {
+      const int h = h0 + wg;
+      const int row = wq * 32 + lane;
+      const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+      const uint32_t tS = tmem + lane_base + (uint32_t)wg * 128u;
+      const uint32_t tO = tmem + lane_base + 256u + (uint32_t)wg * 128u;
+      const int qs = qt * kTile + row;  // logical slot of this query row
+      const int phys_q = qs < p.T ? qs : (qs < p.Pt ? -1 : (qs < p.Pt + p.N ? qs - p.Pt + p.T : -1));
+      const bool q_valid = phys_q >= 0 && phys_q >= p.q_lo && phys_q < p.q_hi;
+      // key slots this row admits beyond the text: [klo, khi)
+      int klo = p.Pt, khi = p.Pt + p.N;
+      if (!p.tile_aligned && phys_q >= p.T) {
+        const int r = (qs - p.Pt) / p.W;
+        klo = p.Pt + max(0, r - p.window_half) * p.W;
+        khi = p.Pt + min(p.H, r + p.window_half + 1) * p.W;
+      }
+      const float sq_row = p.sq ? p.sq[((long long)b * p.Hq + h) * p.nt_scale + qt] : 0.f;
+      const float* sk_row = p.sk ? p.sk + ((long long)b * p.Hkv + g) * p.nt_scale : nullptr;
+      float m = kNegInf, l = 0.f;
+      bool ok = true;
+      if ((p.debug_flags & 1) && wg == 0 && wq == 0) ok = wait_warp(ctl, bar(BAR_NEVER), 0);
+      for (int t = 0; t < n && ok; ++t) {
+        const int e = p.entries[e0 + t];
+        const int kb = e >> 2;
+        ok = wait_warp(ctl, bar(BAR_S + wg), t & 1);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        uint32_t v[128];
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ptx::tmem_ld32(tS + 32u * j, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * j]));
+        ptx::tmem_wait_ld();
+        const int kind = e & 3;
+        // log2-unit score scale; INT8 tiles also carry both block scales (a zero
+        // scale means an all-zero block: any positive multiplier gives score 0)
+        const float mult = (kind & KREA_KIND_INT8) ? fmaxf(p.scale_log2 * sq_row * sk_row[kb], 1e-30f)
+                                                   : p.scale_log2;
+        // admitted key columns of this tile: [0, a1) text, [a2, a3) image window
+        const int s0 = kb * kTile;
+        const int a1 = p.T - s0, a2 = klo - s0, a3 = khi - s0;
+        const bool first = t == 0;
+        if (kind == 0) softmax_tile<BF16, false, false, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d);
+        else if (kind == 1) softmax_tile<BF16, false, true, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d);
+        else if (kind == 2) softmax_tile<BF16, true, false, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d);
+        else softmax_tile<BF16, true, true, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(BAR_P + wg));
+      }
+      if (ok) ok = wait_warp(ctl, bar(BAR_O + wg), 0);
+      if (ok) {
+        ptx::tc_fence_after();
+        const float inv_l = 1.0f / l;
+        const long long tok = q_valid ? phys_q : 0;
+        const uint16_t* grow =
+            p.has_gate ? static_cast<const uint16_t*>(p.gate) + b * p.gate_stride[0] + tok * p.gate_stride[1] +
+                             (long long)h * p.gate_stride[2]
+                       : nullptr;
+        for (int j = 0; j < d / 32; ++j) {
+          uint32_t o[32];
+          __syncwarp();
+          ptx::tmem_ld32(tO + 32u * j, o);
+          ptx::tmem_wait_ld();
+          if (!q_valid) continue;
+          float y[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) y[c] = __uint_as_float(o[c]) * inv_l;
+          if (grow) {
+            const uint4* gp = reinterpret_cast<const uint4*>(grow + 32 * j);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint4 u = gp[v];
+              const uint16_t* ge = reinterpret_cast<const uint16_t*>(&u);
+#pragma unroll
+              for (int c = 0; c < 8; ++c) y[8 * v + c] *= sigmoidf_(h2f<BF16>(ge[c]));
+            }
+          }
+          if (p.out_f32) {
+            float4* op = reinterpret_cast<float4*>(static_cast<float*>(p.out) + b * p.out_stride[0] +
+                                                   tok * p.out_stride[1] + (long long)h * p.out_stride[2] + 32 * j);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) op[v] = make_float4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
+          } else {
+            uint4* op = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + b * p.out_stride[0] +
+                                                 tok * p.out_stride[1] + (long long)h * p.out_stride[2] + 32 * j);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              op[v] = make_uint4(pack2<BF16>(y[8 * v], y[8 * v + 1]), pack2<BF16>(y[8 * v + 2], y[8 * v + 3]),
+                                 pack2<BF16>(y[8 * v + 4], y[8 * v + 5]), pack2<BF16>(y[8 * v + 6], y[8 * v + 7]));
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 9) ptx::tmem_dealloc(tmem, 512);
+}
+
+// ALL_POLY = true sends every exponential through exp2_poly2 (tests of its accuracy).
+template <bool BF16, bool ALL_POLY>
+int launch(const AttnDevParams& p, const void* tq, const void* tk, const void* tv, const void* tq8,
+           const void* tk8, cudaStream_t s) {
+  static int checked = 0;  // 1 = the kernel has the register count the setmaxnreg split needs
+  if (!checked) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<BF16, ALL_POLY>) != cudaSuccess) return KREA_ERR_CUDA;
+    checked = (fa.numRegs == kLaunchRegs) ? 1 : -1;
+  }
+  if (checked != 1) return KREA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(attn_fwd_kernel<BF16, ALL_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)SMEM_ALLOC) != cudaSuccess)
+    return KREA_ERR_CUDA;
+  const long long grid = (long long)p.B * p.Hkv * p.npairs * p.n_slice_tiles;
+  if (grid <= 0 || grid > 0x7fffffffLL) return KREA_ERR_INVALID_ARG;
+  attn_fwd_kernel<BF16, ALL_POLY><<<(unsigned)grid, kThreads, SMEM_ALLOC, s>>>(
+      *static_cast<const CUtensorMap*>(tq), *static_cast<const CUtensorMap*>(tk),
+      *static_cast<const CUtensorMap*>(tv), *static_cast<const CUtensorMap*>(tq8),
+      *static_cast<const CUtensorMap*>(tk8), p);
+  return cudaGetLastError() == cudaSuccess ? KREA_OK : KREA_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_attention(const AttnDevParams& p, const void* tq, const void* tk, const void* tv, const void* tq8,
+                     const void* tk8, bool bf16, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p.debug_flags & 2)
+    return bf16 ? launch<true, true>(p, tq, tk, tv, tq8, tk8, s) : launch<false, true>(p, tq, tk, tv, tq8, tk8, s);
+  return bf16 ? launch<true, false>(p, tq, tk, tv, tq8, tk8, s) : launch<false, false>(p, tq, tk, tv, tq8, tk8, s);
+}
+
+}  // namespace krea

@@ -1,0 +1,179 @@
+/*
+ * krea_attn.h -- C ABI of the Krea 2 bidirectional attention core for B200 (sm_100a).
+ *
+ * One call computes, for every query token t of a [text, image] sequence and every
+ * query head h,
+ *
+ *     out[b,t,h,:] = sigmoid(gate[b,t,h,:]) * sum_{j in A(t)} softmax_j(scale * s(t,j)) * v[b,j,h/rep,:]
+ *
+ * - bidirectional, non-causal attention with one running softmax state per row
+ *   ("Krea 2 TileMix Attention (FP16/INT8 tiles)", section "What it actually patches");
+ * - grouped-query attention resolved inside the kernel: q head h reads kv head
+ *   h / (Hq / Hkv), the repeat_interleave order (same section);
+ * - three modes (krea_mode_t): dense; TileMix, where each 128x128 score tile is
+ *   computed in FP16 or from INT8 codes by a static map (same page, sections
+ *   "What it actually patches" and "The inputs that matter"); and scanline, a
+ *   block-sparse mask in which text is global and an image token sees image tokens
+ *   within window/2 latent rows ("Krea 2 Scanline Attention", section "What the
+ *   mask actually is");
+ * - the sigmoid(gate) multiply of the surrounding block fused into the epilogue;
+ * - query slicing against full K/V ("LayerStream: Krea2 Chunking", section "What the
+ *   node does to the block"): every slice of a 128-aligned query range gives the
+ *   bit-identical rows of the single-slice call.
+ *
+ * Conventions shared by every entry point:
+ * - Tensors are [batch, token, head, head_dim] with head_dim contiguous; the
+ *   (batch, token, head) strides are given in ELEMENTS in krea_attn_params_t.
+ *   q/k/v/gate/out must start on a 16-byte boundary and every stride times the
+ *   element size must be a multiple of 16 bytes.
+ * - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *   never frees or keeps them. The only memory the library owns is its tile-map
+ *   cache (device copies of the block-sparse lists; at most 8 entries per device,
+ *   released by krea_attn_clear_cache()).
+ * - Work is enqueued on `stream` and runs asynchronously; the only blocking step
+ *   is a host-to-device copy when a tile map is built for the first time.
+ * - Every call returns KREA_OK (0) or a negative krea_status_t; no C++ exception
+ *   crosses the ABI. krea_attn_error_string() names a code. Errors detected on
+ *   the device (a bounded wait that ran out) are written to params->status.
+ */
+#ifndef KREA_ATTN_H_
+#define KREA_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KREA_API __attribute__((visibility("default")))
+#else
+#define KREA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KREA_ATTN_ABI_VERSION 1
+#define KREA_ATTN_TILE 128
+
+typedef enum {
+  KREA_MODE_DENSE = 0,     /* every key for every query */
+  KREA_MODE_TILEMIX = 1,   /* per-tile FP16 / INT8 routing by a static map */
+  KREA_MODE_SCANLINE = 2   /* block-sparse scanline mask over 128-token tiles */
+} krea_mode_t;
+
+typedef enum { KREA_F16 = 0, KREA_BF16 = 1, KREA_F32 = 2 } krea_dtype_t;
+
+/* TileMix patterns ("Krea 2 TileMix Attention", section "The inputs that matter"):
+ * zero keeps every tile FP16; band sends a `percentage` share of the left-over
+ * image-image tiles (off the diagonal band) to INT8, farthest from the diagonal
+ * first; one sends all of them to INT8. */
+typedef enum { KREA_PATTERN_ZERO = 0, KREA_PATTERN_BAND = 1, KREA_PATTERN_ONE = 2 } krea_pattern_t;
+
+typedef enum {
+  KREA_OK = 0,
+  KREA_ERR_INVALID_ARG = -1,     /* bad shape, stride, alignment, window, slice or percentage */
+  KREA_ERR_UNSUPPORTED = -2,     /* fp32 inputs, head_dim not 64/128, Hq % Hkv != 0, INT8 with head_dim 64 */
+  KREA_ERR_WORKSPACE = -3,       /* workspace missing or smaller than krea_attn_workspace_bytes() */
+  KREA_ERR_CUDA = -4,            /* a CUDA runtime call or a launch failed */
+  KREA_ERR_DEVICE_TIMEOUT = -5,  /* written to *status: a bounded wait in a kernel ran out */
+  KREA_ERR_DEVICE_BOUNDS = -6,   /* written to *status: a kernel met an out-of-range index */
+  KREA_ERR_NO_DEVICE = -7        /* no CUDA device, or not an sm_100 device */
+} krea_status_t;
+
+/* Kind bits of one tile of a map (krea_attn_get_map). */
+#define KREA_KIND_MASKED 1  /* some key slot of the tile is padding or not admitted */
+#define KREA_KIND_INT8 2    /* the tile's scores come from INT8 codes */
+
+typedef struct {
+  int32_t abi_version;   /* must be KREA_ATTN_ABI_VERSION */
+  int32_t batch;         /* B >= 1 */
+  int32_t num_q_heads;   /* Hq >= 1 */
+  int32_t num_kv_heads;  /* Hkv >= 1, Hq % Hkv == 0 */
+  int32_t head_dim;      /* 64 or 128 (INT8 tiles need 128) */
+  int32_t q_start;       /* first query token of this slice, a multiple of 128 */
+  int32_t q_len;         /* query tokens in this slice; 0 means up to the end */
+  int32_t in_dtype;      /* krea_dtype_t of q, k, v, gate: KREA_F16 or KREA_BF16 */
+  int32_t out_dtype;     /* KREA_F32 or the input dtype */
+  int64_t q_stride[3];   /* (batch, token, head) strides of q, in elements */
+  int64_t k_stride[3];
+  int64_t v_stride[3];
+  int64_t gate_stride[3];
+  int64_t out_stride[3];
+  float softmax_scale;   /* 0 -> 1/sqrt(head_dim) */
+  /* TileMix */
+  int32_t pattern;       /* krea_pattern_t */
+  float percentage;      /* share of left-over image-image tiles sent to INT8, in [0, 1] */
+  int32_t band_blocks;   /* key blocks on each side of the diagonal kept FP16; < 0 -> 2 */
+  int32_t smooth_k;      /* centre K per (batch, kv head, channel) before quantising */
+  int32_t qk_fp32_accumulate; /* accepted and recorded: QK^T always accumulates in fp32 */
+  /* scanline */
+  int32_t window;        /* odd, 1..255: image tokens see image rows within window/2 */
+  int32_t tile_aligned;  /* 1: every valid pair inside an active tile is admitted */
+  int32_t text_pad;      /* text slot size, multiple of 128, >= text_len; 0 -> max(512, ceil128(T)) */
+  /* scratch and status */
+  void* workspace;       /* device memory, krea_attn_workspace_bytes() bytes; TileMix only */
+  size_t workspace_bytes;
+  int32_t* status;       /* optional device int32, zero before the call: a kernel that gives up writes a
+                            negative code; a kernel that finds it nonzero does no work */
+  int64_t debug_wait_limit; /* SM clock cycles a kernel waits on one barrier before giving up; 0 -> 2e9 */
+  int32_t debug_flags;   /* bit 0: one softmax warp waits on a barrier nothing arrives at (tests the bounded wait);
+                            bit 1: every exponential through the FMA-pipe polynomial (tests its accuracy) */
+} krea_attn_params_t;
+
+/* Fill `p` with the defaults for a contiguous [B, L, H, d] layout. */
+KREA_API void krea_attn_default_params(krea_attn_params_t* p, int batch, int num_q_heads, int num_kv_heads,
+                              int head_dim, int text_len, int grid_h, int grid_w);
+
+/* The attention forward. q [B,L,Hq,d], k and v [B,L,Hkv,d], gate [B,L,Hq,d] or NULL,
+ * out [B,L,Hq,d] (only rows q_start .. q_start+q_len-1 are written); L = text_len +
+ * grid_h * grid_w, text tokens first, image tokens row-major on a grid_h x grid_w grid.
+ * mode is a krea_mode_t. TileMix needs params->workspace. */
+KREA_API int krea_attn_fwd(const void* q, const void* k, const void* v, const void* gate, void* out,
+                  int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* params,
+                  void* stream);
+
+/* Bytes of caller-allocated workspace krea_attn_fwd needs (0 if none). */
+KREA_API size_t krea_attn_workspace_bytes(int text_len, int grid_h, int grid_w, int mode,
+                                 const krea_attn_params_t* params);
+
+/* Byte offsets inside the workspace (TileMix) of:
+ *   kc  centred keys k - mean, [B, L, Hkv, d], input dtype (smooth_k only)
+ *   q8  INT8 query codes [B, L, Hq, d];  k8 INT8 key codes [B, L, Hkv, d]
+ *   sq  query scales [B, Hq, nt] f32;    sk key scales [B, Hkv, nt] f32 (nt = ceil(L/128))
+ *   mu  key mean [B, Hkv, d] f32;        part  per-chunk partial sums (f64) */
+typedef struct {
+  size_t kc, q8, k8, sq, sk, mu, part, total;
+} krea_attn_ws_layout_t;
+KREA_API int krea_attn_workspace_layout(int text_len, int grid_h, int grid_w, int mode,
+                               const krea_attn_params_t* params, krea_attn_ws_layout_t* out);
+
+/* Size of the tile map: *n_tiles query tiles (the logical sequence, text slot
+ * included for scanline) and *nnz listed (query tile, key tile) pairs. */
+KREA_API int krea_attn_map_size(int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* params,
+                       int32_t* n_tiles, int32_t* nnz);
+
+/* Copy the tile map into HOST buffers: row_ptr[n_tiles + 1], col[nnz] (key tiles,
+ * ascending per row) and kind[nnz] (KREA_KIND_* bits). `capacity` is the length of
+ * col and kind. Pure host work; needs no GPU. */
+KREA_API int krea_attn_get_map(int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* params,
+                      int32_t* row_ptr, int32_t* col, uint8_t* kind, int32_t capacity);
+
+/* Run only the TileMix quantiser (key mean, centred keys, INT8 codes and scales)
+ * into params->workspace, laid out as krea_attn_workspace_layout() says. */
+KREA_API int krea_attn_quantize(const void* q, const void* k, int text_len, int grid_h, int grid_w,
+                       const krea_attn_params_t* params, void* stream);
+
+/* Release every cached tile map on every device. */
+KREA_API void krea_attn_clear_cache(void);
+
+/* Static text for a krea_status_t. */
+KREA_API const char* krea_attn_error_string(int code);
+
+/* KREA_ATTN_ABI_VERSION of the loaded library. */
+KREA_API int krea_attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KREA_ATTN_H_ */

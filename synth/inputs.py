@@ -18,7 +18,9 @@ layout [batch, tokens, heads, head_dim] (head_dim contiguous), plus the optional
 sigmoid-gate logits [batch, tokens, q_heads, head_dim].
 
 Random numbers come from numpy's PCG64 generator, one independent stream per
-(seed, tensor) pair, drawn in float64 and rounded once to the storage dtype.
+(seed, tensor) pair, drawn in float32 and rounded once to the storage dtype
+(the RMS-normalised, rotated q/k of the 1 MP dense case are computed in fp64
+from those draws before the rounding).
 """
 from __future__ import annotations
 
@@ -74,11 +76,11 @@ class Case:
 
 def _normal(seed: int, stream: str, shape, mean: float = 0.0, std: float = 1.0) -> np.ndarray:
     rng = np.random.default_rng([seed, _STREAM[stream]])
-    x = rng.standard_normal(size=shape, dtype=np.float64)
+    x = rng.standard_normal(size=shape, dtype=np.float32)
     if std != 1.0:
-        x *= std
+        x *= np.float32(std)
     if mean != 0.0:
-        x += mean
+        x += np.float32(mean)
     return x
 
 
@@ -128,8 +130,8 @@ def make_inputs(case: Case, with_gate: Optional[bool] = None):
     v = _normal(case.seed, "v", (B, L, Hkv, d))
     if case.qk_dist == "rms_rope":
         ang = _rope_angles(case)
-        q = _rms_rope(q, ang)
-        k = _rms_rope(k, ang)
+        q = _rms_rope(q.astype(np.float64), ang)
+        k = _rms_rope(k.astype(np.float64), ang)
     elif case.qk_dist == "normal_koffset":
         # a shared per-(kv head, channel) offset ~ N(0.5, 0.1) on every key
         off = _normal(case.seed, "koff", (1, 1, Hkv, d), mean=0.5, std=0.1)

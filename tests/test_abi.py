@@ -1,0 +1,109 @@
+"""The C ABI library: it loads without a GPU, exports every entry point the
+header declares, its params struct matches the binding's, and it rejects bad
+arguments (and, on a machine without an sm_100 GPU, refuses to run) instead of
+falling back to anything."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+import torch
+
+import diffusion_transformer_attention_bidirectional_b200 as K
+from diffusion_transformer_attention_bidirectional_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "krea_attn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"KREA_API\s+[\w\s\*]+?\b(krea_attn_\w+)\s*\(", src)))
+
+
+def test_header_declarations_are_exported():
+    names = declared_functions()
+    assert len(names) >= 10
+    lib = _lib.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, f"binding lacks {n}"
+    out = subprocess.run(["nm", "-D", "--defined-only", str(_lib.LIB_PATH)], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (krea_attn_\w+)", out))
+    assert exported == set(names), exported ^ set(names)
+
+
+def test_params_layout_matches_header():
+    fields = [f for f, _ in _lib.Params._fields_]
+    prog = "#include <stdio.h>\n#include <stddef.h>\n#include \"krea_attn.h\"\nint main(void){\n"
+    prog += 'printf("%zu\\n", sizeof(krea_attn_params_t));\n'
+    for f in fields:
+        prog += f'printf("%zu\\n", offsetof(krea_attn_params_t, {f}));\n'
+    prog += "return 0;}\n"
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(prog)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True).stdout.split()]
+    assert vals[0] == ctypes.sizeof(_lib.Params)
+    for f, off in zip(fields, vals[1:]):
+        assert getattr(_lib.Params, f).offset == off, f
+
+
+def test_error_strings():
+    for code in range(0, -8, -1):
+        s = _lib.lib().krea_attn_error_string(code).decode()
+        assert s and s != "unknown error"
+    assert _lib.lib().krea_attn_abi_version() == 1
+
+
+def _fwd(p, T=16, H=8, W=8, mode=0, ptr=1 << 20):
+    return _lib.lib().krea_attn_fwd(ptr, ptr, ptr, None, ptr, T, H, W, mode, ctypes.byref(p), None)
+
+
+def test_invalid_arguments_rejected_without_gpu():
+    p = K.make_params(1, 4, 1, 64, 16, 8, 8, in_dtype="f16")
+    bad = [
+        dict(num_q_heads=6, num_kv_heads=4, code=-2),  # Hq % Hkv
+        dict(head_dim=96, code=-2),
+        dict(in_dtype=2, code=-2),                     # fp32 input
+        dict(out_dtype=1, code=-1),                    # bf16 out for f16 in
+        dict(q_start=64, code=-1),
+        dict(abi_version=7, code=-1),
+        dict(batch=0, code=-1),
+    ]
+    for b in bad:
+        q = K.make_params(1, 4, 1, 64, 16, 8, 8, in_dtype="f16")
+        code = b.pop("code")
+        for f, v in b.items():
+            setattr(q, f, v)
+        assert _fwd(q) == code, b
+    assert _fwd(p, ptr=(1 << 20) + 8) == -1             # misaligned pointer
+    p.q_stride[2] = 60                                    # 120 bytes: not a 16-byte multiple
+    assert _fwd(p) == -1
+    w = K.make_params(1, 4, 1, 64, 16, 8, 8, window=4)
+    assert _fwd(w, mode=2) == -1                          # even window
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
+def test_no_device_is_an_error_not_a_fallback():
+    p = K.make_params(1, 4, 1, 64, 16, 8, 8, in_dtype="f16")
+    assert _fwd(p) == _lib.ERR_NO_DEVICE
+    with pytest.raises(ValueError):
+        q = torch.zeros(1, 80, 4, 64, dtype=torch.float16)
+        K.attention(q, q[:, :, :1], q[:, :, :1], text_len=16, grid_h=8, grid_w=8)
+
+
+def test_workspace_sizes():
+    p = K.make_params(1, 48, 12, 128, 512, 128, 128, in_dtype="f16")
+    lay = K.workspace_layout(512, 128, 128, p)
+    L = 512 + 128 * 128
+    assert lay["q8"] >= L * 12 * 128 * 2          # centred keys first
+    assert lay["k8"] - lay["q8"] >= L * 48 * 128
+    assert lay["total"] == K.workspace_bytes("tilemix", 512, 128, 128, p)
+    assert K.workspace_bytes("dense", 512, 128, 128, p) == 0
+    for k in ("kc", "q8", "k8", "sq", "sk", "mu", "part"):
+        assert lay[k] % 256 == 0
