@@ -265,6 +265,108 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int
   l += (s0 + s1) + (s2 + s3);
 }
 
+// The single thread that issues every tcgen05.mma of the CTA. Descriptors are
+// built once and advanced by constant adds (the 14-bit start-address field
+// cannot carry: shared addresses stay below 256 KB), and every K loop is
+// unrolled, so that issuing keeps ahead of the tensor core (one 128x128x16 MMA
+// completes every 64 cycles).
+template <bool BF16, int D>
+__device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base, uint32_t tmem, int e0, int n,
+                                           int nh, const Ctl& ctl) {
+  auto bar = [&](int i) { return base + SM_BAR + 8u * (uint32_t)i; };
+  constexpr uint32_t ab = BF16 ? 1u : 0u;
+  constexpr uint32_t ID_QK = ptx::idesc(1, ab, 0, 0, 128, 128);
+  constexpr uint32_t ID_QK8 = ptx::idesc(2, 1, 0, 0, 128, 128);
+  constexpr uint32_t ID_PV = ptx::idesc(1, ab, 0, 1, D, 128);
+  // low words of the shared-memory descriptors (start address >> 4 sits in bits 0..13)
+  const uint32_t dq = ptx::sdesc_lo(base + SM_Q, 16);      // Q of head i: + i * 32 KB
+  const uint32_t dq8 = ptx::sdesc_lo(base + SM_Q8, 16);    // Q codes of head i: + i * 16 KB
+  const uint32_t dk = ptx::sdesc_lo(base + SM_SLOT, 16);   // slot s, K-major: + s * 32 KB
+  const uint32_t dv = ptx::sdesc_lo(base + SM_SLOT, kBox); // slot s, MN-major (V)
+  auto qk = [&](int i, int kind, uint32_t slot) {
+    const uint32_t dS = tmem + (uint32_t)i * 128u;
+    const uint32_t kd = dk + slot * (kTileBytes >> 4);
+    if (kind & KREA_KIND_INT8) {
+      const uint32_t qd = dq8 + (uint32_t)i * (kBox >> 4);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)  // K = 32 bytes per step
+        ptx::mma_i8_ss_lo(dS, qd + 2 * k, kd + 2 * k, ID_QK8, k > 0);
+    } else {
+      const uint32_t qd = dq + (uint32_t)i * (kTileBytes >> 4);
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {  // K = 16 elements (32 bytes) per step
+        constexpr uint32_t kb4 = kBox >> 4;
+        const uint32_t off = (uint32_t)(k >> 2) * kb4 + (uint32_t)(k & 3) * 2u;
+        ptx::mma_f16_ss_lo(dS, qd + off, kd + off, ID_QK, k > 0);
+      }
+    }
+  };
+  auto pv = [&](int i, uint32_t slot, uint32_t acc) {
+    const uint32_t dO = tmem + 256u + (uint32_t)i * 128u;
+    const uint32_t aP = tmem + (uint32_t)i * 128u;
+    const uint32_t vd = dv + slot * (kTileBytes >> 4);
+    ptx::mma_f16_ts_lo(dO, aP, vd, ID_PV, acc);
+#pragma unroll
+    for (int k = 1; k < 8; ++k)  // 16 keys per step: 8 TMEM columns of P, 16 rows of V (2 KB)
+      ptx::mma_f16_ts_lo(dO, aP + 8u * k, vd + 128u * k, ID_PV, 1);
+  };
+  bool ok = wait1(ctl, bar(BAR_Q), 0);
+  uint32_t it = 0;
+  if (ok) {
+    ptx::tc_fence_after();
+    ok = wait1(ctl, bar(BAR_FULL + 0), 0);
+  }
+  if (ok) {
+    ptx::tc_fence_after();
+    const int kind0 = p.entries[e0] & 3;
+    int e_next = n > 1 ? p.entries[e0 + 1] : 0;  // map entries are read one tile ahead
+    for (int i = 0; i < nh; ++i) {
+      qk(i, kind0, 0);
+      ptx::tc_commit(bar(BAR_S + i));
+    }
+    ptx::tc_commit(bar(BAR_EMPTY + 0));
+    it = 1;
+    for (int t = 0; t < n && ok; ++t) {
+      const uint32_t slot_v = it % kSlots;
+      ok = wait1(ctl, bar(BAR_FULL + slot_v), (it / kSlots) & 1);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      ++it;
+      const bool has_next = t + 1 < n;
+      const uint32_t slot_k = it % kSlots;
+      const int kind_next = e_next & 3;
+      if (t + 2 < n) e_next = p.entries[e0 + t + 2];
+      for (int i = 0; i < nh && ok; ++i) {
+        ok = wait1(ctl, bar(BAR_P + i), t & 1);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        pv(i, slot_v, t > 0 ? 1u : 0u);
+        if (has_next) {
+          if (i == 0) {
+            ok = wait1(ctl, bar(BAR_FULL + slot_k), (it / kSlots) & 1);
+            if (!ok) break;
+            ptx::tc_fence_after();
+          }
+          qk(i, kind_next, slot_k);
+          ptx::tc_commit(bar(BAR_S + i));
+        }
+      }
+      if (!ok) break;
+      ptx::tc_commit(bar(BAR_EMPTY + slot_v));
+      if (has_next) {
+        ptx::tc_commit(bar(BAR_EMPTY + slot_k));
+        ++it;
+      }
+    }
+  }
+  if (ok)
+    for (int i = 0; i < nh; ++i) ptx::tc_commit(bar(BAR_O + i));
+  // every MMA this thread issued finishes before TMEM is freed, also when a
+  // softmax warp gave up waiting on O
+  ptx::tc_commit(bar(BAR_DRAIN));
+  wait_drain(bar(BAR_DRAIN), 0);
+}
+
 // ---------------------------------------------------------------------------
 template <bool BF16, bool ALL_POLY>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -378,90 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t ab = BF16 ? 1u : 0u;
-      const uint32_t id_qk = ptx::idesc(1, ab, 0, 0, 128, 128);
-      const uint32_t id_qk8 = ptx::idesc(2, 1, 0, 0, 128, 128);
-      const uint32_t id_pv = ptx::idesc(1, ab, 0, 1, (uint32_t)d, 128);
-      const int ksteps = d / 16;
-      auto issue_qk = [&](int i, int kind, uint32_t slot) {
-        const uint32_t dS = tmem + (uint32_t)i * 128u;
-        const uint32_t kaddr = base + SM_SLOT + slot * kTileBytes;
-        if (kind & KREA_KIND_INT8) {
-          const uint32_t qaddr = base + SM_Q8 + (uint32_t)i * kBox;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)  // K = 32 bytes per step
-            ptx::mma_i8_ss(dS, ptx::sdesc(qaddr + 32 * k, 16, 1024), ptx::sdesc(kaddr + 32 * k, 16, 1024),
-                           id_qk8, k > 0);
-        } else {
-          const uint32_t qaddr = base + SM_Q + (uint32_t)i * kTileBytes;
-          for (int k = 0; k < ksteps; ++k) {  // K = 16 elements (32 bytes) per step
-            const uint32_t off = (uint32_t)(k >> 2) * kBox + (uint32_t)(k & 3) * 32;
-            ptx::mma_f16_ss(dS, ptx::sdesc(qaddr + off, 16, 1024), ptx::sdesc(kaddr + off, 16, 1024), id_qk,
-                            k > 0);
-          }
-        }
-      };
-      auto issue_pv = [&](int i, uint32_t slot, bool acc) {
-        const uint32_t dO = tmem + 256u + (uint32_t)i * 128u;
-        const uint32_t aP = tmem + (uint32_t)i * 128u;
-        const uint32_t vaddr = base + SM_SLOT + slot * kTileBytes;
-#pragma unroll
-        for (int k = 0; k < 8; ++k)  // 16 keys per step: 8 TMEM columns of P, 16 V rows
-          ptx::mma_f16_ts(dO, aP + 8u * k, ptx::sdesc(vaddr + 2048u * k, kBox, 1024), id_pv, (acc || k > 0));
-      };
-      bool ok = wait1(ctl, bar(BAR_Q), 0);
-      uint32_t it = 0;
-      if (ok) {
-        ptx::tc_fence_after();
-        ok = wait1(ctl, bar(BAR_FULL + 0), 0);
-      }
-      if (ok) {
-        ptx::tc_fence_after();
-        const int kind0 = p.entries[e0] & 3;
-        for (int i = 0; i < nh; ++i) {
-          issue_qk(i, kind0, 0);
-          ptx::tc_commit(bar(BAR_S + i));
-        }
-        ptx::tc_commit(bar(BAR_EMPTY + 0));
-        it = 1;
-        for (int t = 0; t < n && ok; ++t) {
-          const uint32_t slot_v = it % kSlots;
-          ok = wait1(ctl, bar(BAR_FULL + slot_v), (it / kSlots) & 1);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          ++it;
-          const bool has_next = t + 1 < n;
-          const uint32_t slot_k = it % kSlots;
-          const int kind_next = has_next ? (p.entries[e0 + t + 1] & 3) : 0;
-          for (int i = 0; i < nh && ok; ++i) {
-            ok = wait1(ctl, bar(BAR_P + i), t & 1);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            issue_pv(i, slot_v, t > 0);
-            if (has_next) {
-              if (i == 0) {
-                ok = wait1(ctl, bar(BAR_FULL + slot_k), (it / kSlots) & 1);
-                if (!ok) break;
-                ptx::tc_fence_after();
-              }
-              issue_qk(i, kind_next, slot_k);
-              ptx::tc_commit(bar(BAR_S + i));
-            }
-          }
-          if (!ok) break;
-          ptx::tc_commit(bar(BAR_EMPTY + slot_v));
-          if (has_next) {
-            ptx::tc_commit(bar(BAR_EMPTY + slot_k));
-            ++it;
-          }
-        }
-      }
-      if (ok)
-        for (int i = 0; i < nh; ++i) ptx::tc_commit(bar(BAR_O + i));
-      // every MMA this thread issued finishes before TMEM is freed, also when a
-      // softmax warp gave up waiting on O
-      ptx::tc_commit(bar(BAR_DRAIN));
-      wait_drain(bar(BAR_DRAIN), 0);
+      if (d == 128) mma_thread<BF16, 128>(p, base, tmem, e0, n, nh, ctl);
+      else mma_thread<BF16, 64>(p, base, tmem, e0, n, nh, ctl);
     }
   }
   } else {
@@ -489,8 +509,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = kNegInf, l = 0.f;
       bool ok = true;
       if ((p.debug_flags & 1) && wg == 0 && wq == 0) ok = wait_warp(ctl, bar(BAR_NEVER), 0);
+      int e_pre = p.entries[e0];
       for (int t = 0; t < n && ok; ++t) {
-        const int e = p.entries[e0 + t];
+        const int e = e_pre;
+        if (t + 1 < n) e_pre = p.entries[e0 + t + 1];  // read one tile ahead
         const int kb = e >> 2;
         ok = wait_warp(ctl, bar(BAR_S + wg), t & 1);
         if (!ok) break;

@@ -198,6 +198,44 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo_bytes, uin
   return d;
 }
 
+// The same descriptor split in two 32-bit words: the low word holds the start
+// address and LBO (changes per operand), the high word SBO = 1024, the version
+// and the swizzle mode (a compile-time constant).
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t addr, uint32_t lbo_bytes) {
+  return ((addr & 0x3FFFF) >> 4) | (((lbo_bytes >> 4) & 0x3FFF) << 16);
+}
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+
+// D (+)= A * B^T with both operands in shared memory, descriptors given by their low words.
+__device__ __forceinline__ void mma_f16_ss_lo(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                              uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "mov.b64 da, {%1, %5};\n\tmov.b64 db, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accum), "n"(kDescHi)
+      : "memory");
+}
+__device__ __forceinline__ void mma_i8_ss_lo(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
+                                             uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "mov.b64 da, {%1, %5};\n\tmov.b64 db, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], da, db, %3, p;\n\t}" ::"r"(d),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accum), "n"(kDescHi)
+      : "memory");
+}
+// D (+)= A[tmem] * B[smem], B descriptor by its low word.
+__device__ __forceinline__ void mma_f16_ts_lo(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
+                                              uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "mov.b64 db, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accum), "n"(kDescHi)
+      : "memory");
+}
+
 // Instruction descriptor of kind::f16 / kind::i8 MMAs.
 //   c_fmt: 1 = f32, 2 = s32; ab_fmt: f16 0 / bf16 1, or s8 1; majors: 0 = K, 1 = MN.
 __host__ __device__ constexpr uint32_t idesc(uint32_t c_fmt, uint32_t ab_fmt, uint32_t a_major,
