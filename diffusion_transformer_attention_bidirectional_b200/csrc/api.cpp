@@ -423,9 +423,9 @@ int krea_attn_fwd(const void* q, const void* k, const void* v, const void* gate,
   for (int i = 0; i < 3; ++i) kc_stride[i] = p->k_stride[i];
   const float* sq = nullptr;
   const float* sk = nullptr;
-  CUtensorMap tm_q, tm_k, tm_v, tm_q8, tm_k8;
-  std::memset(&tm_q8, 0, sizeof(tm_q8));
-  std::memset(&tm_k8, 0, sizeof(tm_k8));
+  AttnMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  CUtensorMap &tm_q = maps.q, &tm_k = maps.k, &tm_v = maps.v, &tm_q8 = maps.q8, &tm_k8 = maps.k8;
   if (use_int8 || centred) {
     rc = run_quantize(q, k, g, p, use_int8, stream);
     if (rc != KREA_OK) return rc;
@@ -452,6 +452,11 @@ int krea_attn_fwd(const void* q, const void* k, const void* v, const void* gate,
   if (rc == KREA_OK) rc = make_tmap(&tm_k, k_src, tdt, es, d, Hkv, g.L, B, kc_stride, box);
   if (rc == KREA_OK) rc = make_tmap(&tm_v, v, tdt, es, d, Hkv, g.L, B, p->v_stride, box);
   if (rc != KREA_OK) return rc;
+  // epilogue maps: gate (16-bit, 64 per 128-byte row) and out (fp32: 32, 16-bit: 64)
+  bool tma_out = make_tmap(&maps.out, out,
+                           p->out_dtype == KREA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : tdt, oes, d, Hq, g.L, B,
+                           p->out_stride, p->out_dtype == KREA_F32 ? 32 : 64) == KREA_OK;
+  if (tma_out && gate) tma_out = make_tmap(&maps.gate, gate, tdt, es, d, Hq, g.L, B, p->gate_stride, box) == KREA_OK;
 
   AttnDevParams ap;
   std::memset(&ap, 0, sizeof(ap));
@@ -494,9 +499,10 @@ int krea_attn_fwd(const void* q, const void* k, const void* v, const void* gate,
   ap.scale_log2 = scale * 1.4426950408889634f;
   ap.has_gate = gate != nullptr;
   ap.out_f32 = p->out_dtype == KREA_F32;
+  ap.tma_out = tma_out ? 1 : 0;
   ap.wait_limit = p->debug_wait_limit > 0 ? p->debug_wait_limit : (long long)2000000000LL;
   ap.debug_flags = p->debug_flags;
-  return launch_attention(ap, &tm_q, &tm_k, &tm_v, &tm_q8, &tm_k8, bf16, stream);
+  return launch_attention(ap, maps, bf16, stream);
 }
 
 void krea_attn_clear_cache(void) {

@@ -64,7 +64,10 @@ constexpr uint32_t SM_SLOT = 98304;    // kSlots x 32 KB
 constexpr uint32_t SM_BAR = SM_SLOT + kSlots * kTileBytes;
 constexpr int BAR_Q = 0, BAR_FULL = 1, BAR_EMPTY = BAR_FULL + kSlots, BAR_S = BAR_EMPTY + kSlots,
               BAR_P = BAR_S + 2, BAR_O = BAR_P + 2, BAR_DRAIN = BAR_O + 2, BAR_NEVER = BAR_DRAIN + 1,
-              N_BARS = BAR_NEVER + 1;
+              BAR_QFREE = BAR_NEVER + 1,  // the last QK^T finished: the Q area may be reused
+              BAR_GATE = BAR_QFREE + 1,   // gate tiles landed in the Q area
+              BAR_EPI = BAR_GATE + 1,     // 2: all 128 rows of head i staged for the TMA store
+              N_BARS = BAR_EPI + 2;
 constexpr uint32_t SM_TMEM_PTR = SM_BAR + 8 * N_BARS;
 constexpr uint32_t SM_ABORT = SM_TMEM_PTR + 4;
 constexpr uint32_t SMEM_USED = SM_BAR + 256;
@@ -72,6 +75,12 @@ constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // slack to align the base to
 static_assert(8 * N_BARS + 8 <= 256, "barrier block overflow");
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 constexpr long long kDrainLimit = 4000000000LL;
+// Pairs of exponentials computed by the FMA-pipe polynomial: bit (i % 8) of
+// kPolyMask for pair i. Measured on B200 inside this kernel: every offload
+// fraction tried (1/4, 3/8) was slower than none, since the softmax warps are
+// then bound by issue and latency rather than by the exponential unit; the
+// polynomial stays available (debug_flags bit 1 runs every exponential on it).
+constexpr uint32_t kPolyMask = 0x00u;
 constexpr float kNegInf = -INFINITY;
 
 struct Ctl {
@@ -143,7 +152,11 @@ __device__ __forceinline__ float h2f(uint16_t u) {
   }
 }
 
-__device__ __forceinline__ float sigmoidf_(float x) { return __frcp_rn(1.0f + __expf(-x)); }
+// sigmoid(x) = 1 / (1 + 2^(-x log2 e)): two exponential-unit operations; x -> -inf
+// gives 1/inf = 0, x -> +inf gives 1.
+__device__ __forceinline__ float sigmoidf_(float x) {
+  return ptx::rcp_approx(1.0f + ptx::ex2(x * -1.4426950408889634f));
+}
 
 // 2^x on the FMA pipe for a pair of values, so that part of the exponentials
 // leaves the MUFU unit (whose 16 results per clock per SM would otherwise bound
@@ -162,9 +175,7 @@ __device__ __forceinline__ void exp2_poly2(float& a, float& b) {
   const uint64_t x = ptx::f2(a, b);
   const uint64_t j = ptx::add2(x, ptx::f2(kRound, kRound));
   const uint64_t n = ptx::add2(j, ptx::f2(-kRound, -kRound));
-  float n0, n1;
-  ptx::unf2(n, n0, n1);
-  const uint64_t f = ptx::add2(x, ptx::f2(-n0, -n1));
+  const uint64_t f = ptx::fma2(n, ptx::f2(-1.0f, -1.0f), x);  // x - n
   uint64_t p;
   if constexpr (BF16) {
     p = ptx::fma2(ptx::f2(0.055417872965335846f, 0.055417872965335846f), f,
@@ -206,13 +217,15 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int
     if constexpr (MASKED) r = ((c < a1) || (c >= a2 && c < a3)) ? r : kNegInf;
     v[c] = __float_as_uint(r);
   }
-  float mx0 = kNegInf, mx1 = kNegInf;
+  float mx0 = kNegInf, mx1 = kNegInf, mx2 = kNegInf, mx3 = kNegInf;
 #pragma unroll
-  for (int c = 0; c < 128; c += 4) {
+  for (int c = 0; c < 128; c += 8) {  // four independent chains: short latency
     mx0 = ptx::max3(mx0, __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
     mx1 = ptx::max3(mx1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+    mx2 = ptx::max3(mx2, __uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
+    mx3 = ptx::max3(mx3, __uint_as_float(v[c + 6]), __uint_as_float(v[c + 7]));
   }
-  const float m_tile = fmaxf(mx0, mx1) * mult;  // mult > 0
+  const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * mult;  // mult > 0
   const float m_new = fmaxf(m, m_tile);
   if (first) {
     m = m_new;
@@ -247,7 +260,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int
       const uint64_t x = ptx::fma2(ptx::f2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), mult2, negm2);
       float p0, p1;
       ptx::unf2(x, p0, p1);
-      if (ALL_POLY || (i & 3) == 3) {
+      if (ALL_POLY || ((kPolyMask >> (i % 8)) & 1u)) {
         exp2_poly2<BF16>(p0, p1);
       } else {
         p0 = ptx::ex2(p0);
@@ -325,6 +338,7 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
       ptx::tc_commit(bar(BAR_S + i));
     }
     ptx::tc_commit(bar(BAR_EMPTY + 0));
+    if (n == 1) ptx::tc_commit(bar(BAR_QFREE));
     it = 1;
     for (int t = 0; t < n && ok; ++t) {
       const uint32_t slot_v = it % kSlots;
@@ -352,6 +366,7 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
         }
       }
       if (!ok) break;
+      if (t + 2 == n) ptx::tc_commit(bar(BAR_QFREE));  // the last QK^T has been issued
       ptx::tc_commit(bar(BAR_EMPTY + slot_v));
       if (has_next) {
         ptx::tc_commit(bar(BAR_EMPTY + slot_k));
@@ -370,9 +385,7 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
 // ---------------------------------------------------------------------------
 template <bool BF16, bool ALL_POLY>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q8,
-                    const __grid_constant__ CUtensorMap tm_k8, const __grid_constant__ AttnDevParams p) {
+    attn_fwd_kernel(const __grid_constant__ AttnMaps tm, const __grid_constant__ AttnDevParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -412,6 +425,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::mbar_init(bar(BAR_DRAIN), 1);
     ptx::mbar_init(bar(BAR_NEVER), 1);
+    ptx::mbar_init(bar(BAR_QFREE), 1);
+    ptx::mbar_init(bar(BAR_GATE), 1);
+    ptx::mbar_init(bar(BAR_EPI + 0), 128);
+    ptx::mbar_init(bar(BAR_EPI + 1), 128);
     *abort_flag = 0;
     ptx::fence_barrier_init();
     ptx::fence_proxy_async_smem();
@@ -426,25 +443,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_ptr;
   const int nh = p.nh;
   const int d = p.d;
+  // Staged epilogue (gate prefetched by TMA, output written by TMA stores) when the
+  // tile's physical rows are exactly its query rows and all lie in the slice:
+  // no text padding inside the tile; rows past L are clipped by the TMA unit.
+  const int qrow0 = tile_row0(qt, p);
+  const int s0q = qt * kTile;
+  const bool staged = p.tma_out && ((s0q + kTile <= p.T) || (s0q >= p.Pt) || (p.T == p.Pt)) &&
+                      qrow0 >= p.q_lo && min(qrow0 + kTile, p.L) <= p.q_hi;
 
   if (warp >= 8) {
   ptx::regs_dec<kOtherRegs>();  // the whole third warpgroup
   if (warp == 8) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
-      ptx::prefetch_tmap(&tm_q);
-      ptx::prefetch_tmap(&tm_k);
-      ptx::prefetch_tmap(&tm_v);
+      ptx::prefetch_tmap(&tm.q);
+      ptx::prefetch_tmap(&tm.k);
+      ptx::prefetch_tmap(&tm.v);
       bool has_int8 = false;
       for (int t = 0; t < n; ++t) has_int8 |= (p.entries[e0 + t] & KREA_KIND_INT8) != 0;
       const int nbox = d / 64;
-      const int qrow0 = tile_row0(qt, p);
       ptx::mbar_arrive_expect_tx(bar(BAR_Q), nh * nbox * kBox + (has_int8 ? nh * kBox : 0));
       for (int i = 0; i < nh; ++i) {
         for (int x = 0; x < nbox; ++x)
-          ptx::tma_load_4d(base + SM_Q + i * kTileBytes + x * kBox, &tm_q, bar(BAR_Q), x * 64, h0 + i, qrow0, b);
-        if (has_int8) ptx::tma_load_4d(base + SM_Q8 + i * kBox, &tm_q8, bar(BAR_Q), 0, h0 + i, qrow0, b);
+          ptx::tma_load_4d(base + SM_Q + i * kTileBytes + x * kBox, &tm.q, bar(BAR_Q), x * 64, h0 + i, qrow0, b);
+        if (has_int8) ptx::tma_load_4d(base + SM_Q8 + i * kBox, &tm.q8, bar(BAR_Q), 0, h0 + i, qrow0, b);
       }
+      if (staged && p.has_gate)  // warm L2 with the gate tiles the epilogue will need
+        for (int i = 0; i < nh; ++i)
+          for (int x = 0; x < nbox; ++x) ptx::tma_prefetch_l2_4d(&tm.gate, x * 64, h0 + i, qrow0, b);
       uint32_t it = 0;
       for (int t = 0; t < n; ++t) {
         const int e = p.entries[e0 + t];
@@ -455,11 +481,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t dst = base + SM_SLOT + slot * kTileBytes;
         if (e & KREA_KIND_INT8) {
           ptx::mbar_arrive_expect_tx(bar(BAR_FULL + slot), kBox);
-          ptx::tma_load_4d(dst, &tm_k8, bar(BAR_FULL + slot), 0, g, krow0, b);
+          ptx::tma_load_4d(dst, &tm.k8, bar(BAR_FULL + slot), 0, g, krow0, b);
         } else {
           ptx::mbar_arrive_expect_tx(bar(BAR_FULL + slot), nbox * kBox);
           for (int x = 0; x < nbox; ++x)
-            ptx::tma_load_4d(dst + x * kBox, &tm_k, bar(BAR_FULL + slot), x * 64, g, krow0, b);
+            ptx::tma_load_4d(dst + x * kBox, &tm.k, bar(BAR_FULL + slot), x * 64, g, krow0, b);
         }
         ++it;
         // V tile
@@ -468,12 +494,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         dst = base + SM_SLOT + slot * kTileBytes;
         ptx::mbar_arrive_expect_tx(bar(BAR_FULL + slot), nbox * kBox);
         for (int x = 0; x < nbox; ++x)
-          ptx::tma_load_4d(dst + x * kBox, &tm_v, bar(BAR_FULL + slot), x * 64, g, krow0, b);
+          ptx::tma_load_4d(dst + x * kBox, &tm.v, bar(BAR_FULL + slot), x * 64, g, krow0, b);
         ++it;
+      }
+      // gate tiles of the staged epilogue go into the Q area once the last QK^T is done
+      bool gate_issued = false;
+      if (staged && p.has_gate && it == 2u * (uint32_t)n && wait1(ctl, bar(BAR_QFREE), 0)) {
+        ptx::mbar_arrive_expect_tx(bar(BAR_GATE), nh * nbox * kBox);
+        for (int i = 0; i < nh; ++i)
+          for (int x = 0; x < nbox; ++x)
+            ptx::tma_load_4d(base + SM_Q + i * kTileBytes + x * kBox, &tm.gate, bar(BAR_GATE), x * 64, h0 + i,
+                             qrow0, b);
+        gate_issued = true;
       }
       // Every copy this thread started lands before the CTA may exit (already
       // true on the normal path, where the MMA thread consumed them all).
       wait_drain(bar(BAR_Q), 0);
+      if (gate_issued) wait_drain(bar(BAR_GATE), 0);
       for (uint32_t j = (it > kSlots ? it - kSlots : 0); j < it; ++j)
         wait_drain(bar(BAR_FULL + j % kSlots), (j / kSlots) & 1);
     }
@@ -541,7 +578,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) ptx::mbar_arrive(bar(BAR_P + wg));
       }
       if (ok) ok = wait_warp(ctl, bar(BAR_O + wg), 0);
-      if (ok) {
+      if (ok && staged && p.has_gate) ok = wait_warp(ctl, bar(BAR_GATE), 0);
+      if (ok && staged) {
+        // Staged epilogue: the gate row comes from the Q area (TMA-loaded, 64 values per
+        // 128-byte swizzled row), out = O / l * sigmoid(gate) goes to the free K/V slots
+        // in the 128-byte swizzled layout of the out map, then one thread stores by TMA.
+        ptx::tc_fence_after();
+        const float inv_l = 1.0f / l;
+        const uint32_t obytes = p.out_f32 ? 4u : 2u;
+        const uint32_t gbase = SM_Q + (uint32_t)wg * kTileBytes;
+        const uint32_t stage = SM_SLOT + (uint32_t)wg * (uint32_t)(kTile * d) * obytes;
+        const uint32_t rsw = (uint32_t)(row & 7), rofs = (uint32_t)row * 128u;
+        for (int j = 0; j < d / 32; ++j) {
+          uint32_t o[32];
+          __syncwarp();
+          ptx::tmem_ld32(tO + 32u * j, o);
+          ptx::tmem_wait_ld();
+          float y[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) y[c] = __uint_as_float(o[c]) * inv_l;
+          if (p.has_gate) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {  // columns 32j + 8v ..: box j/2, 16-byte piece (j%2)*4 + v
+              const uint32_t q = (uint32_t)((j & 1) * 4 + v);
+              const uint4 u = *reinterpret_cast<const uint4*>(sb + gbase + (uint32_t)(j >> 1) * kBox + rofs +
+                                                               ((q ^ rsw) << 4));
+              const uint16_t* ge = reinterpret_cast<const uint16_t*>(&u);
+#pragma unroll
+              for (int c = 0; c < 8; ++c) y[8 * v + c] *= sigmoidf_(h2f<BF16>(ge[c]));
+            }
+          }
+          if (p.out_f32) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)  // box j holds columns 32j .. 32j+31
+              *reinterpret_cast<float4*>(sb + stage + (uint32_t)j * kBox + rofs + (((uint32_t)v ^ rsw) << 4)) =
+                  make_float4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
+          } else {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {  // box j/2 holds columns 64(j/2) ..; piece (j%2)*4 + v
+              const uint32_t q = (uint32_t)((j & 1) * 4 + v);
+              *reinterpret_cast<uint4*>(sb + stage + (uint32_t)(j >> 1) * kBox + rofs + ((q ^ rsw) << 4)) =
+                  make_uint4(pack2<BF16>(y[8 * v], y[8 * v + 1]), pack2<BF16>(y[8 * v + 2], y[8 * v + 3]),
+                             pack2<BF16>(y[8 * v + 4], y[8 * v + 5]), pack2<BF16>(y[8 * v + 6], y[8 * v + 7]));
+            }
+          }
+        }
+        ptx::fence_proxy_async_smem();  // make the rows visible to the TMA unit
+        ptx::mbar_arrive(bar(BAR_EPI + wg));
+        if (wq == 0 && lane == 0 && wait1(ctl, bar(BAR_EPI + wg), 0)) {
+          const int wbox = p.out_f32 ? 32 : 64;
+          for (int x = 0; x < d / wbox; ++x)
+            ptx::tma_store_4d(&tm.out, base + stage + (uint32_t)x * kBox, x * wbox, h, qrow0, b);
+          ptx::bulk_commit();
+          ptx::bulk_wait_read0();  // shared memory must outlive the store's reads
+        }
+      } else if (ok) {
         ptx::tc_fence_after();
         const float inv_l = 1.0f / l;
         const long long tok = q_valid ? phys_q : 0;
@@ -594,8 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ALL_POLY = true sends every exponential through exp2_poly2 (tests of its accuracy).
 template <bool BF16, bool ALL_POLY>
-int launch(const AttnDevParams& p, const void* tq, const void* tk, const void* tv, const void* tq8,
-           const void* tk8, cudaStream_t s) {
+int launch(const AttnDevParams& p, const AttnMaps& maps, cudaStream_t s) {
   static int checked = 0;  // 1 = the kernel has the register count the setmaxnreg split needs
   if (!checked) {
     cudaFuncAttributes fa;
@@ -608,21 +698,16 @@ int launch(const AttnDevParams& p, const void* tq, const void* tk, const void* t
     return KREA_ERR_CUDA;
   const long long grid = (long long)p.B * p.Hkv * p.npairs * p.n_slice_tiles;
   if (grid <= 0 || grid > 0x7fffffffLL) return KREA_ERR_INVALID_ARG;
-  attn_fwd_kernel<BF16, ALL_POLY><<<(unsigned)grid, kThreads, SMEM_ALLOC, s>>>(
-      *static_cast<const CUtensorMap*>(tq), *static_cast<const CUtensorMap*>(tk),
-      *static_cast<const CUtensorMap*>(tv), *static_cast<const CUtensorMap*>(tq8),
-      *static_cast<const CUtensorMap*>(tk8), p);
+  attn_fwd_kernel<BF16, ALL_POLY><<<(unsigned)grid, kThreads, SMEM_ALLOC, s>>>(maps, p);
   return cudaGetLastError() == cudaSuccess ? KREA_OK : KREA_ERR_CUDA;
 }
 
 }  // namespace
 
-int launch_attention(const AttnDevParams& p, const void* tq, const void* tk, const void* tv, const void* tq8,
-                     const void* tk8, bool bf16, void* stream) {
+int launch_attention(const AttnDevParams& p, const AttnMaps& maps, bool bf16, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (p.debug_flags & 2)
-    return bf16 ? launch<true, true>(p, tq, tk, tv, tq8, tk8, s) : launch<false, true>(p, tq, tk, tv, tq8, tk8, s);
-  return bf16 ? launch<true, false>(p, tq, tk, tv, tq8, tk8, s) : launch<false, false>(p, tq, tk, tv, tq8, tk8, s);
+  if (p.debug_flags & 2) return bf16 ? launch<true, true>(p, maps, s) : launch<false, true>(p, maps, s);
+  return bf16 ? launch<true, false>(p, maps, s) : launch<false, false>(p, maps, s);
 }
 
 }  // namespace krea

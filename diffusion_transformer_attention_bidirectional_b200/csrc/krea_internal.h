@@ -2,6 +2,8 @@
 // Krea 2 attention core. Not part of the public ABI (include/krea_attn.h is).
 #pragma once
 
+#include <cuda.h>
+
 #include <cstddef>
 #include <cstdint>
 #include <vector>
@@ -63,6 +65,7 @@ struct AttnDevParams {
   int nt_scale;        // tiles per (batch, head) in sq / sk
   float scale_log2;    // softmax scale * log2(e)
   int has_gate, out_f32;
+  int tma_out;         // out (and gate, when given) have TMA maps: staged epilogue allowed
   long long wait_limit;
   int debug_flags;
 };
@@ -92,8 +95,10 @@ WsLayout workspace_layout(int B, int L, int Hq, int Hkv, int d, int in_bytes, in
 
 // Kernel launchers (attn_sm100.cu, quant.cu). Return KREA_OK or KREA_ERR_CUDA.
 int launch_quantize(const QuantDevParams& p, bool bf16, void* stream);
-int launch_attention(const AttnDevParams& p, const void* tmap_q, const void* tmap_k,
-                     const void* tmap_v, const void* tmap_q8, const void* tmap_k8, bool bf16,
-                     void* stream);
+// TMA descriptors of one attention call (passed to the kernel as one parameter).
+struct alignas(64) AttnMaps {
+  CUtensorMap q, k, v, q8, k8, gate, out;
+};
+int launch_attention(const AttnDevParams& p, const AttnMaps& maps, bool bf16, void* stream);
 
 }  // namespace krea
