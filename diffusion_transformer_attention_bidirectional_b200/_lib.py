@@ -25,6 +25,7 @@ ERR_CUDA = -4
 ERR_DEVICE_TIMEOUT = -5
 ERR_DEVICE_BOUNDS = -6
 ERR_NO_DEVICE = -7
+ERR_TOO_LARGE = -8
 
 KIND_MASKED = 1
 KIND_INT8 = 2
@@ -78,6 +79,7 @@ _I = ctypes.c_int
 SIGNATURES = {
     "krea_attn_default_params": (None, [_P, _I, _I, _I, _I, _I, _I, _I]),
     "krea_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _P, _VP]),
+    "krea_attn_fwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _P, _VP]),
     "krea_attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _P]),
     "krea_attn_workspace_layout": (_I, [_I, _I, _I, _I, _P, ctypes.POINTER(WsLayout)]),
     "krea_attn_map_size": (_I, [_I, _I, _I, _I, _P, ctypes.POINTER(ctypes.c_int32),

@@ -272,6 +272,7 @@ const char* krea_attn_error_string(int code) {
     case KREA_ERR_DEVICE_TIMEOUT: return "device: a bounded wait ran out";
     case KREA_ERR_DEVICE_BOUNDS: return "device: index out of range";
     case KREA_ERR_NO_DEVICE: return "no sm_100 CUDA device";
+    case KREA_ERR_TOO_LARGE: return "shape needs more scratch than the fixed 64 MiB array of krea_attn_fwd_noalloc";
     default: return "unknown error";
   }
 }

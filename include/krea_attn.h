@@ -77,7 +77,8 @@ typedef enum {
   KREA_ERR_CUDA = -4,            /* a CUDA runtime call or a launch failed */
   KREA_ERR_DEVICE_TIMEOUT = -5,  /* written to *status: a bounded wait in a kernel ran out */
   KREA_ERR_DEVICE_BOUNDS = -6,   /* written to *status: a kernel met an out-of-range index */
-  KREA_ERR_NO_DEVICE = -7        /* no CUDA device, or not an sm_100 device */
+  KREA_ERR_NO_DEVICE = -7,       /* no CUDA device, or not an sm_100 device */
+  KREA_ERR_TOO_LARGE = -8        /* krea_attn_fwd_noalloc: the shape needs more scratch than its fixed array */
 } krea_status_t;
 
 /* Kind bits of one tile of a map (krea_attn_get_map). */
@@ -162,6 +163,25 @@ KREA_API int krea_attn_get_map(int text_len, int grid_h, int grid_w, int mode, c
  * into params->workspace, laid out as krea_attn_workspace_layout() says. */
 KREA_API int krea_attn_quantize(const void* q, const void* k, int text_len, int grid_h, int grid_w,
                        const krea_attn_params_t* params, void* stream);
+
+/* The same attention as krea_attn_fwd, for callers that cannot allocate device
+ * memory while they run (an arena or pool that forbids cudaMalloc/cudaFree, which
+ * synchronise the device; a host framework that owns all device memory; a serving
+ * loop that must not block on the allocator). It allocates, caches and frees
+ * nothing: the tile map and the TileMix workspace live in one fixed 64 MiB array
+ * in device memory declared by the library, held on every GPU that loads the
+ * library until the process exits; params->workspace is ignored. Shapes whose
+ * map plus workspace exceed 64 MiB return KREA_ERR_TOO_LARGE before any launch
+ * (a 48/12-head TileMix call fits up to about 1 MP; dense and scanline calls fit
+ * far beyond 4 MP). All calls share the array, so calls whose GPU work overlaps
+ * (two streams, or two threads on one device) race and must not be issued; calls
+ * on one stream are ordered. Each call rewrites everything it reads, nothing
+ * needs clearing. The first call on a device looks up the array's device address;
+ * make it before any CUDA graph capture on that device. The pages describe no
+ * counterpart of this entry point. */
+KREA_API int krea_attn_fwd_noalloc(const void* q, const void* k, const void* v, const void* gate, void* out,
+                                   int text_len, int grid_h, int grid_w, int mode,
+                                   const krea_attn_params_t* params, void* stream);
 
 /* Release every cached tile map on every device. */
 KREA_API void krea_attn_clear_cache(void);

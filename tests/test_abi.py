@@ -54,7 +54,7 @@ def test_params_layout_matches_header():
 
 
 def test_error_strings():
-    for code in range(0, -8, -1):
+    for code in range(0, -9, -1):
         s = _lib.lib().krea_attn_error_string(code).decode()
         assert s and s != "unknown error"
     assert _lib.lib().krea_attn_abi_version() == 1
