@@ -38,6 +38,23 @@ WORKLOAD = ("krea2_4mp_attention_step: dense CFG pair B=2 bf16+gate sliced 4096 
 TILE = 128
 
 
+def roofline_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
+    or None once the kernel source differs from the one the counters came from."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "attn_fwd_roofline.json")
+    src = os.path.join(ROOT, "diffusion_transformer_attention_bidirectional_b200", "csrc", "attn_sm100.cu")
+    try:
+        rec = json.load(open(path))
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except (OSError, ValueError):
+        return None, None
+    if rec.get("kernel_source_sha256") != digest:
+        return None, rec
+    return rec.get("dram_bytes_per_launch"), rec
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -121,6 +138,20 @@ def make_call(case, K, bufs, ws, status):
     return launches, n_kernels
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest value of x over all ranks (timings are reported as the max)."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs the same step (weak scaling), time is the max."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -136,7 +167,7 @@ class ClockSampler:
         try:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.file, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -244,13 +275,9 @@ def run_ours(args, rank, world, device):
     clocks = sampler.stop()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during timing")
-    step_ms = sum(per_step) / len(per_step)
-    if world > 1:
-        t = torch.tensor([step_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = max_over_ranks(sum(per_step) / len(per_step), world, device)
     total_flops = sum(flops)
-    value = world * total_flops / (step_ms * 1e-3) / 1e12
+    value = job_throughput(total_flops, world, step_ms)
 
     # e2e through the public API with host buffers: pinned H2D of every input,
     # the step, D2H of every output, all inside the timed span
@@ -270,17 +297,14 @@ def run_ours(args, rank, world, device):
             hout.copy_(dout, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(device)
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * total_flops / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, device)
+    e2e_value = job_throughput(total_flops, world, e2e_ms)
 
     # roofline of the dominant kernel: the attention kernel on the dense variant
     # (its launches are attention kernels only), algorithmic FLOPs / event time
     dense_attn_ms = attn_dense_ms / args.steps
     achieved = flops[0] / (dense_attn_ms * 1e-3) / 1e12
+    traffic, traffic_rec = roofline_traffic()
     names = [c.name for c in cases]
     variants = {}
     for i, c in enumerate(cases):
@@ -295,18 +319,25 @@ def run_ours(args, rank, world, device):
             n8 = int(((kind & 2) > 0).sum())
             f8 = flops[i] * (n8 / len(kind)) / 2
             pk = flops[i] / ((flops[i] - f8) / P["bf16"] + f8 / (2 * P["bf16"]))
+        pks = pk * P["bf16_sustained"] / P["bf16"]
         variants[names[i]] = {"ms": round(ms, 4), "tflops": round(tf, 1), "peak_tflops": round(pk, 1),
-                              "frac_of_peak": round(tf / pk, 4), "gflop": round(flops[i] / 1e9, 1)}
+                              "frac_of_peak": round(tf / pk, 4), "frac_of_sustained_peak": round(tf / pks, 4),
+                              "gflop": round(flops[i] / 1e9, 1)}
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "global_batch": world * 4, "seq_len": cases[0].seq_len,
                    "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MB write)"},
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": P["bf16"], "unit": "TFLOP/s",
-                     "frac": round(achieved / P["bf16"], 4), "traffic": None,
+        # the attention launches run back to back inside a ~0.5 s timed loop, where the
+        # power cap engages: the sustained measured peak is the denominator, the burst
+        # fraction is reported beside it
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": P["bf16_sustained"],
+                     "unit": "TFLOP/s", "frac": round(achieved / P["bf16_sustained"], 4),
+                     "frac_of_burst_peak": round(achieved / P["bf16"], 4), "traffic": traffic,
                      "kernel": "attn_fwd_kernel<bf16> (dense CFG pair, 5 slices)",
-                     "peak_source": f"{P['source']} bf16 burst"},
+                     "traffic_source": (traffic_rec or {}).get("launch"),
+                     "peak_source": f"{P['source']} bf16 sustained (burst {P['bf16']})"},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": kernels * args.steps,
@@ -381,7 +412,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

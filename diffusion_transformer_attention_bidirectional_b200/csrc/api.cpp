@@ -206,7 +206,7 @@ namespace krea {
 WsLayout workspace_layout(int B, int L, int Hq, int Hkv, int d, int in_bytes, int smooth_k) {
   WsLayout w;
   const int nt = (L + kTile - 1) / kTile;
-  w.chunk_tokens = 64;
+  w.chunk_tokens = 128;
   w.n_chunks = (L + w.chunk_tokens - 1) / w.chunk_tokens;
   size_t off = 0;
   w.kc = off;

@@ -268,3 +268,22 @@ def test_polynomial_exp2_path(dtype):
     compare(c, out, q, k, v, g)
     base = gpu_run(c, q, k, v, g)
     assert float((out - base).abs().max()) < 4e-3
+
+
+def test_head_shards_equal_full_call():
+    # the multi-GPU split: each rank's call on views of its kv heads (here run one
+    # after the other on one GPU) fills exactly the rows of the full call
+    from diffusion_transformer_attention_bidirectional_b200 import shard
+
+    c = S.Case("shards", 1, 48, 12, 128, 256, 24, 24, dtype="bf16", mode="scanline", seed=51, window=7,
+               gate=True)
+    q, k, v, g = (t.cuda() for t in S.make_inputs(c))
+    full = K.attention(q, k, v, g, text_len=c.text_len, grid_h=c.grid_h, grid_w=c.grid_w, mode="scanline",
+                       window=7)
+    out = torch.full_like(full, float("nan"))
+    for rank in range(3):
+        qs, ks, vs, gs, os_ = shard.shard_views(q, k, v, g, out, rank, 3)
+        K.attention(qs, ks, vs, gs, text_len=c.text_len, grid_h=c.grid_h, grid_w=c.grid_w, mode="scanline",
+                    window=7, out=os_)
+    torch.cuda.synchronize()
+    assert torch.equal(out, full)
