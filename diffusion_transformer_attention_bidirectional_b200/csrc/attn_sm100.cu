@@ -391,10 +391,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sb = smem_raw + (base - raw);
 
-  // work item: (batch, kv head, head pair, query tile), query tile fastest
+  // work item: (batch, kv head, head pair, query tile), query tile fastest; the
+  // slice's first n_heavy query tiles (the longest map rows) come first for every
+  // (batch, kv head, head pair), then the rest
   int idx = blockIdx.x;
-  const int qt = p.tile_begin + idx % p.n_slice_tiles;
-  idx /= p.n_slice_tiles;
+  const int heavy_ctas = p.B * p.Hkv * p.npairs * p.n_heavy;
+  int ql;
+  if (idx < heavy_ctas) {
+    ql = idx % p.n_heavy;
+    idx /= p.n_heavy;
+  } else {
+    idx -= heavy_ctas;
+    const int n_light = p.n_slice_tiles - p.n_heavy;
+    ql = p.n_heavy + idx % n_light;
+    idx /= n_light;
+  }
+  const int qt = p.tile_begin + ql;
   const int pair = idx % p.npairs;
   idx /= p.npairs;
   const int g = idx % p.Hkv;

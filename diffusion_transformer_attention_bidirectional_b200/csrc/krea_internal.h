@@ -61,6 +61,7 @@ struct AttnDevParams {
   int B, Hq, Hkv, d, rep, nh, npairs;
   int T, N, Pt, L, W, H, window_half, tile_aligned;
   int n_tiles, tile_begin, n_slice_tiles;
+  int n_heavy;         // the slice's first n_heavy query tiles have the longest rows: launched first
   int q_lo, q_hi;      // physical query rows written: [q_lo, q_hi)
   int nt_scale;        // tiles per (batch, head) in sq / sk
   float scale_log2;    // softmax scale * log2(e)

@@ -24,6 +24,7 @@
 // cudaGetSymbolAddress (the array's name in host code is only a host-side
 // stand-in, not a device address); make that first call before any CUDA graph
 // capture on that device.
+#include <algorithm>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -259,6 +260,14 @@ extern "C" int krea_attn_fwd_noalloc(const void* q, const void* k, const void* v
   auto slot_of = [&](int t) { return t < g.T ? t : t - g.T + g.Pt; };
   ap.tile_begin = slot_of(ap.q_lo) / kTile;
   ap.n_slice_tiles = slot_of(ap.q_hi - 1) / kTile - ap.tile_begin + 1;
+  // Scanline: text query rows see every key tile, image rows only the text and their
+  // window, so the text tiles' CTAs go first and no long row starts in the last wave.
+  {
+    const int text_tiles = (g.T + kTile - 1) / kTile;
+    ap.n_heavy = mode == KREA_MODE_SCANLINE
+                     ? std::max(0, std::min(ap.tile_begin + ap.n_slice_tiles, text_tiles) - ap.tile_begin)
+                     : 0;
+  }
   ap.nt_scale = (g.L + kTile - 1) / kTile;
   const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt((float)d);
   ap.scale_log2 = scale * 1.4426950408889634f;
