@@ -67,7 +67,8 @@ constexpr int BAR_Q = 0, BAR_FULL = 1, BAR_EMPTY = BAR_FULL + kSlots, BAR_S = BA
               BAR_QFREE = BAR_NEVER + 1,  // the last QK^T finished: the Q area may be reused
               BAR_GATE = BAR_QFREE + 1,   // gate tiles landed in the Q area
               BAR_EPI = BAR_GATE + 1,     // 2: all 128 rows of head i staged for the TMA store
-              N_BARS = BAR_EPI + 2;
+              BAR_Q8 = BAR_EPI + 2,       // INT8 query codes landed (rows with INT8 tiles only)
+              N_BARS = BAR_Q8 + 1;
 constexpr uint32_t SM_TMEM_PTR = SM_BAR + 8 * N_BARS;
 constexpr uint32_t SM_ABORT = SM_TMEM_PTR + 4;
 constexpr uint32_t SMEM_USED = SM_BAR + 256;
@@ -324,11 +325,20 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
       ptx::mma_f16_ts_lo(dO, aP + 8u * k, vd + 128u * k, ID_PV, 1);
   };
   bool ok = wait1(ctl, bar(BAR_Q), 0);
+  bool q8_ready = false;  // the INT8 query codes are awaited before the first INT8 tile
+  auto need_q8 = [&](int kind) {
+    if (!(kind & KREA_KIND_INT8) || q8_ready) return true;
+    if (!wait1(ctl, bar(BAR_Q8), 0)) return false;
+    ptx::tc_fence_after();
+    q8_ready = true;
+    return true;
+  };
   uint32_t it = 0;
   if (ok) {
     ptx::tc_fence_after();
     ok = wait1(ctl, bar(BAR_FULL + 0), 0);
   }
+  if (ok) ok = need_q8(p.entries[e0] & 3);
   if (ok) {
     ptx::tc_fence_after();
     const int kind0 = p.entries[e0] & 3;
@@ -357,7 +367,7 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
         pv(i, slot_v, t > 0 ? 1u : 0u);
         if (has_next) {
           if (i == 0) {
-            ok = wait1(ctl, bar(BAR_FULL + slot_k), (it / kSlots) & 1);
+            ok = wait1(ctl, bar(BAR_FULL + slot_k), (it / kSlots) & 1) && need_q8(kind_next);
             if (!ok) break;
             ptx::tc_fence_after();
           }
@@ -439,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(bar(BAR_NEVER), 1);
     ptx::mbar_init(bar(BAR_QFREE), 1);
     ptx::mbar_init(bar(BAR_GATE), 1);
+    ptx::mbar_init(bar(BAR_Q8), 1);
     ptx::mbar_init(bar(BAR_EPI + 0), 128);
     ptx::mbar_init(bar(BAR_EPI + 1), 128);
     *abort_flag = 0;
@@ -471,15 +482,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::prefetch_tmap(&tm.q);
       ptx::prefetch_tmap(&tm.k);
       ptx::prefetch_tmap(&tm.v);
-      bool has_int8 = false;
-      for (int t = 0; t < n; ++t) has_int8 |= (p.entries[e0 + t] & KREA_KIND_INT8) != 0;
       const int nbox = d / 64;
-      ptx::mbar_arrive_expect_tx(bar(BAR_Q), nh * nbox * kBox + (has_int8 ? nh * kBox : 0));
-      for (int i = 0; i < nh; ++i) {
+      ptx::mbar_arrive_expect_tx(bar(BAR_Q), nh * nbox * kBox);
+      for (int i = 0; i < nh; ++i)
         for (int x = 0; x < nbox; ++x)
           ptx::tma_load_4d(base + SM_Q + i * kTileBytes + x * kBox, &tm.q, bar(BAR_Q), x * 64, h0 + i, qrow0, b);
-        if (has_int8) ptx::tma_load_4d(base + SM_Q8 + i * kBox, &tm.q8, bar(BAR_Q), 0, h0 + i, qrow0, b);
-      }
       if (staged && p.has_gate)  // warm L2 with the gate tiles the epilogue will need
         for (int i = 0; i < nh; ++i)
           for (int x = 0; x < nbox; ++x) ptx::tma_prefetch_l2_4d(&tm.gate, x * 64, h0 + i, qrow0, b);
@@ -531,6 +538,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       if (d == 128) mma_thread<BF16, 128>(p, base, tmem, e0, n, nh, ctl);
       else mma_thread<BF16, 64>(p, base, tmem, e0, n, nh, ctl);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------- INT8 query codes
+    // Off the producer's path: scanning the row's map entries would delay Q and K_0.
+    if (lane == 0) {
+      bool has_int8 = false;
+      for (int t = 0; t < n; ++t) has_int8 |= (p.entries[e0 + t] & KREA_KIND_INT8) != 0;
+      if (has_int8) {
+        ptx::prefetch_tmap(&tm.q8);
+        ptx::mbar_arrive_expect_tx(bar(BAR_Q8), nh * kBox);
+        for (int i = 0; i < nh; ++i)
+          ptx::tma_load_4d(base + SM_Q8 + i * kBox, &tm.q8, bar(BAR_Q8), 0, h0 + i, qrow0, b);
+        wait_drain(bar(BAR_Q8), 0);  // the copy lands before the CTA may exit
+      }
     }
   }
   } else {
