@@ -94,6 +94,27 @@ def get_map(mode: str, text_len: int, grid_h: int, grid_w: int, params: Optional
     return row_ptr, col[:nnz], kind[:nnz]
 
 
+def get_map_device(mode: str, text_len: int, grid_h: int, grid_w: int, params: Optional[Params] = None,
+                   device=None, capacity: Optional[int] = None, status: Optional[torch.Tensor] = None, **opts):
+    """The tile map built on the GPU: (row_ptr[n_tiles+1] int32, col[capacity] int32,
+    kind[capacity] uint8) device tensors; the first row_ptr[-1] entries are the map."""
+    if params is None:
+        params = make_params(1, 1, 1, 128, text_len, grid_h, grid_w, **opts)
+    device = torch.device(device if device is not None else "cuda")
+    nt, _ = map_size(mode, text_len, grid_h, grid_w, params)
+    cap = nt * nt if capacity is None else capacity
+    row_ptr = torch.empty(nt + 1, dtype=torch.int32, device=device)
+    col = torch.empty(max(cap, 1), dtype=torch.int32, device=device)
+    kind = torch.empty(max(cap, 1), dtype=torch.uint8, device=device)
+    if status is not None:
+        params.status = status.data_ptr()
+    stream = torch.cuda.current_stream(device).cuda_stream
+    check(lib().krea_attn_build_map_device(text_len, grid_h, grid_w, _lib.MODE[mode], ctypes.byref(params),
+                                           row_ptr.data_ptr(), col.data_ptr(), kind.data_ptr(), cap, stream),
+          "build_map_device")
+    return row_ptr, col, kind
+
+
 def _check_inputs(*ts):
     for t in ts:
         if t is not None and not t.is_cuda:

@@ -86,6 +86,7 @@ SIGNATURES = {
                                 ctypes.POINTER(ctypes.c_int32)]),
     "krea_attn_get_map": (_I, [_I, _I, _I, _I, _P, _VP, _VP, _VP, ctypes.c_int32]),
     "krea_attn_quantize": (_I, [_VP, _VP, _I, _I, _I, _P, _VP]),
+    "krea_attn_build_map_device": (_I, [_I, _I, _I, _I, _P, _VP, _VP, _VP, ctypes.c_int32, _VP]),
     "krea_attn_clear_cache": (None, []),
     "krea_attn_error_string": (ctypes.c_char_p, [_I]),
     "krea_attn_abi_version": (_I, []),

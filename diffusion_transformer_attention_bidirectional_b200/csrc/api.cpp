@@ -308,6 +308,17 @@ int krea_attn_get_map(int text_len, int grid_h, int grid_w, int mode, const krea
   return KREA_OK;
 }
 
+int krea_attn_build_map_device(int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* params,
+                               int32_t* row_ptr, int32_t* col, uint8_t* kind, int32_t capacity, void* stream) {
+  Geometry g;
+  int rc = make_geometry(text_len, grid_h, grid_w, mode, params, &g);
+  if (rc != KREA_OK) return rc;
+  if (!row_ptr || !col || !kind || capacity < 0) return KREA_ERR_INVALID_ARG;
+  rc = check_device();
+  if (rc != KREA_OK) return rc;
+  return launch_build_map(g, row_ptr, nullptr, col, kind, capacity, params->status, stream);
+}
+
 size_t krea_attn_workspace_bytes(int text_len, int grid_h, int grid_w, int mode,
                                  const krea_attn_params_t* p) {
   if (mode != KREA_MODE_TILEMIX || check_common(p) != KREA_OK) return 0;

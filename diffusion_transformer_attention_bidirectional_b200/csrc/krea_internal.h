@@ -43,6 +43,12 @@ struct HostMap {
 // Builds a map (tilemap.cpp). Returns KREA_OK or an error code.
 int build_map(const Geometry& g, HostMap* out);
 
+// Builds the map on the device (mapgen.cu): row_ptr[n_tiles + 1], and either packed
+// entries ((key tile << 2) | kind, packed != nullptr) or col / kind arrays. Nothing
+// is written past `capacity` entries; an overflow is reported through `status`.
+int launch_build_map(const Geometry& g, int32_t* row_ptr, int32_t* packed, int32_t* col, uint8_t* kind,
+                     int capacity, int32_t* status, void* stream);
+
 // Resolves and validates the geometry of a call.
 int make_geometry(int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* p,
                   Geometry* g);

@@ -159,6 +159,19 @@ KREA_API int krea_attn_map_size(int text_len, int grid_h, int grid_w, int mode, 
 KREA_API int krea_attn_get_map(int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* params,
                       int32_t* row_ptr, int32_t* col, uint8_t* kind, int32_t capacity);
 
+/* Build the same tile map on the DEVICE, asynchronously on `stream`, into device
+ * buffers row_ptr[n_tiles + 1], col[capacity] and kind[capacity], laid out as
+ * krea_attn_get_map's (map rules: "Krea 2 Scanline Attention", section "What the
+ * mask actually is"; "Krea 2 TileMix Attention (FP16/INT8 tiles)", sections "What
+ * it actually patches" and "The inputs that matter"). n_tiles comes from
+ * krea_attn_map_size, and capacity = n_tiles * n_tiles always suffices. row_ptr is
+ * always written (row_ptr[n_tiles] = nnz); when nnz > capacity, col and kind are
+ * left untouched and params->status, if set, receives KREA_ERR_DEVICE_BOUNDS.
+ * No host work beyond validation, no allocation, no copy. */
+KREA_API int krea_attn_build_map_device(int text_len, int grid_h, int grid_w, int mode,
+                                        const krea_attn_params_t* params, int32_t* row_ptr, int32_t* col,
+                                        uint8_t* kind, int32_t capacity, void* stream);
+
 /* Run only the TileMix quantiser (key mean, centred keys, INT8 codes and scales)
  * into params->workspace, laid out as krea_attn_workspace_layout() says. */
 KREA_API int krea_attn_quantize(const void* q, const void* k, int text_len, int grid_h, int grid_w,
