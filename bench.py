@@ -17,6 +17,7 @@ problems, no collective on the data path); rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -214,7 +215,7 @@ def run_ours(args, rank, world, device):
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
     status = torch.zeros(1, dtype=torch.int32, device=device)
-    host, dev_bufs, calls, flops, kernels = [], [], [], [], 0
+    host, dev_bufs, calls, flops, kernels, workspaces = [], [], [], [], 0, []
     for c in cases:
         q, k, v, g = S.make_inputs(c)
         hb = [t.pin_memory() if t is not None else None for t in (q, k, v, g)]
@@ -227,6 +228,7 @@ def run_ours(args, rank, world, device):
             ws = torch.empty(K.workspace_bytes("tilemix", c.text_len, c.grid_h, c.grid_w, p), dtype=torch.uint8,
                              device=device)
         launches, nk = make_call(c, K, (*db, out), ws, status)
+        workspaces.append(ws)
         host.append((hb, torch.empty(out.shape, dtype=out.dtype, pin_memory=True)))
         dev_bufs.append((db, out))
         calls.append(launches)
@@ -321,6 +323,37 @@ def run_ours(args, rank, world, device):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, device)
     e2e_value = job_throughput(total_flops, world, e2e_ms)
 
+    # Checks of the pages' claims, outside the timed step (median of 5, L2 flushed):
+    # TileMix band against the same call with every tile FP16 (pattern "zero"),
+    # beside the speedup the map predicts when INT8 halves the QK^T half of a tile.
+    comparisons = {}
+    for i, c in enumerate(cases):
+        if c.mode != "tilemix" or c.pattern == "zero" or args.no_comparisons:
+            continue
+        db, dout = dev_bufs[i]
+        zero_calls, _ = make_call(dataclasses.replace(c, pattern="zero"), K, (*db, dout), workspaces[i], status)
+        times = {"band": [], "zero": []}
+        for _ in range(5):
+            for name, fns in (("band", calls[i]), ("zero", zero_calls)):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for fn in fns:
+                    fn()
+                b.record(stream)
+                torch.cuda.synchronize(device)
+                times[name].append(a.elapsed_time(b))
+        med = {k: sorted(v)[len(v) // 2] for k, v in times.items()}
+        rp, col, kind = K.get_map("tilemix", c.text_len, c.grid_h, c.grid_w, pattern=c.pattern,
+                                  percentage=c.percentage, band_blocks=c.band_blocks)
+        n8 = int(((kind & 2) > 0).sum())
+        comparisons[f"{c.name}_vs_pattern_zero"] = {
+            "band_ms": round(med["band"], 4), "zero_ms": round(med["zero"], 4),
+            "speedup": round(med["zero"] / med["band"], 4),
+            "modelled_speedup": round(2 * len(kind) / (2 * (len(kind) - n8) + 1.5 * n8), 4)}
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during the comparisons")
+
     # roofline of the dominant kernel: the attention kernel on the dense variant
     # (its launches are attention kernels only), algorithmic FLOPs / event time
     dense_attn_ms = attn_dense_ms / args.steps
@@ -363,7 +396,14 @@ def run_ours(args, rank, world, device):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": kernels * args.steps,
         "variants": variants,
+        "comparisons": comparisons,
     }
+    dense_tf = next((v["tflops"] for n, v in variants.items() if "cfg_pair" in n), None)
+    for n, v in variants.items():
+        if dense_tf and n.startswith("scanline"):
+            # scanline visits only active tiles: at dense efficiency its time would
+            # scale with its admitted pairs, i.e. this ratio would be 1
+            comparisons[f"{n}_efficiency_vs_dense"] = round(v["tflops"] / dense_tf, 4)
     if clocks:
         res["clocks"] = clocks
     return res
@@ -437,6 +477,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-comparisons", action="store_true",
+                    help="skip the band-vs-zero timing after the timed steps (launch-list captures)")
     ap.add_argument("--case", default=None,
                     help="profile one workload alone (a synth.inputs case or a step variant name)")
     args = ap.parse_args()
