@@ -193,6 +193,18 @@ def test_config_scanline_1mp(T, H, W):
     compare(c, out, q, k, v, g, rows=rows, heads=[0, 5, 47])
 
 
+def test_config_scanline_1mp_token_rule():
+    # tile_aligned off: each image query admits exactly the keys within five rows
+    # (64-token rows, two per tile, so boundary tiles become masked tiles)
+    c = S.scanline_1mp()
+    c.tile_aligned = False
+    q, k, v, g = S.make_inputs(c)
+    out = gpu_run(c, q, k, v, g)
+    L = c.seq_len
+    rows = np.unique(np.r_[np.arange(0, 4), np.arange(508, 700), np.arange(2500, 2600), np.arange(L - 130, L)])
+    compare(c, out, q, k, v, g, rows=rows, heads=[0, 7, 47])
+
+
 def test_config_tilemix_band_4mp():
     c = S.tilemix_band_4mp()
     q, k, v, g = S.make_inputs(c)
