@@ -115,6 +115,69 @@ def get_map_device(mode: str, text_len: int, grid_h: int, grid_w: int, params: O
     return row_ptr, col, kind
 
 
+def rope_positions(text_len: int, grid_h: int, grid_w: int, device=None) -> torch.Tensor:
+    """[L, 3] int32 rotary positions: text token t at (t, 0, 0), image token (r, c) at (0, r, c)."""
+    L = text_len + grid_h * grid_w
+    pos = torch.zeros(L, 3, dtype=torch.int32)
+    pos[:text_len, 0] = torch.arange(text_len, dtype=torch.int32)
+    img = torch.arange(grid_h * grid_w, dtype=torch.int32)
+    pos[text_len:, 1] = img // max(grid_w, 1)
+    pos[text_len:, 2] = img % max(grid_w, 1)
+    return pos.to(device) if device is not None else pos
+
+
+def rope_params(head_dim: int = 128, axes_dim=None, theta: Optional[float] = None,
+                eps: Optional[float] = None) -> _lib.RopeParams:
+    r = _lib.RopeParams()
+    lib().krea_attn_default_rope(ctypes.byref(r), head_dim)
+    if axes_dim is not None:
+        for i in range(3):
+            r.axes_dim[i] = int(axes_dim[i])
+    if theta is not None:
+        r.theta = float(theta)
+    if eps is not None:
+        r.eps = float(eps)
+    return r
+
+
+def rope_table(pos: torch.Tensor, rope: Optional[_lib.RopeParams] = None, head_dim: int = 128,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """(cos, sin) table [L, n_pairs, 2] fp32 on pos's device, for krea_attn_qk_prologue."""
+    _check_inputs(pos)
+    rope = rope if rope is not None else rope_params(head_dim)
+    pos = pos.to(torch.int32).contiguous()
+    n_pairs = sum(rope.axes_dim) // 2
+    table = torch.empty(pos.shape[0], n_pairs, 2, dtype=torch.float32, device=pos.device)
+    check(lib().krea_attn_rope_table(pos.data_ptr(), pos.shape[0], ctypes.byref(rope), table.data_ptr(),
+                                     _stream_ptr(stream, pos.device)), "rope_table")
+    return table
+
+
+def qk_prologue(x: torch.Tensor, table: torch.Tensor, gamma: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, rope: Optional[_lib.RopeParams] = None,
+                with_codes: bool = False, stream: Optional[torch.cuda.Stream] = None):
+    """rope(rmsnorm(x)) for x [B, L, H, d] fp16/bf16 (out may be x). With with_codes,
+    also returns the INT8 codes [B, L, H, d] and block scales [B, H, ceil(L/128)]."""
+    _check_inputs(x, table, gamma, out)
+    B, L, H, d = x.shape
+    rope = rope if rope is not None else rope_params(d)
+    y = out if out is not None else torch.empty_like(x)
+    codes = scales = None
+    if with_codes:
+        codes = torch.empty(B, L, H, d, dtype=torch.int8, device=x.device)
+        scales = torch.empty(B, H, -(-L // 128), dtype=torch.float32, device=x.device)
+    dt = {torch.float16: _lib.DTYPE["f16"], torch.bfloat16: _lib.DTYPE["bf16"]}.get(x.dtype, _lib.DTYPE["f32"])
+    xs = (ctypes.c_int64 * 3)(*x.stride()[:3])
+    ys = (ctypes.c_int64 * 3)(*y.stride()[:3])
+    g = gamma.to(torch.float32).contiguous() if gamma is not None else None
+    check(lib().krea_attn_qk_prologue(x.data_ptr(), y.data_ptr(), g.data_ptr() if g is not None else None,
+                                      table.data_ptr(), B, L, H, d, dt, xs, ys, ctypes.byref(rope),
+                                      codes.data_ptr() if codes is not None else None,
+                                      scales.data_ptr() if scales is not None else None,
+                                      _stream_ptr(stream, x.device)), "qk_prologue")
+    return (y, codes, scales) if with_codes else y
+
+
 def _check_inputs(*ts):
     for t in ts:
         if t is not None and not t.is_cuda:

@@ -66,6 +66,12 @@ class Params(ctypes.Structure):
     ]
 
 
+class RopeParams(ctypes.Structure):
+    """krea_rope_params_t."""
+
+    _fields_ = [("axes_dim", ctypes.c_int32 * 3), ("theta", ctypes.c_float), ("eps", ctypes.c_float)]
+
+
 class WsLayout(ctypes.Structure):
     """krea_attn_ws_layout_t."""
 
@@ -87,6 +93,10 @@ SIGNATURES = {
     "krea_attn_get_map": (_I, [_I, _I, _I, _I, _P, _VP, _VP, _VP, ctypes.c_int32]),
     "krea_attn_quantize": (_I, [_VP, _VP, _I, _I, _I, _P, _VP]),
     "krea_attn_build_map_device": (_I, [_I, _I, _I, _I, _P, _VP, _VP, _VP, ctypes.c_int32, _VP]),
+    "krea_attn_default_rope": (None, [ctypes.POINTER(RopeParams), _I]),
+    "krea_attn_rope_table": (_I, [_VP, _I, ctypes.POINTER(RopeParams), _VP, _VP]),
+    "krea_attn_qk_prologue": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int64),
+                                   ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(RopeParams), _VP, _VP, _VP]),
     "krea_attn_clear_cache": (None, []),
     "krea_attn_error_string": (ctypes.c_char_p, [_I]),
     "krea_attn_abi_version": (_I, []),

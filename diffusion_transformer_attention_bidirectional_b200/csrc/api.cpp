@@ -319,6 +319,75 @@ int krea_attn_build_map_device(int text_len, int grid_h, int grid_w, int mode, c
   return launch_build_map(g, row_ptr, nullptr, col, kind, capacity, params->status, stream);
 }
 
+void krea_attn_default_rope(krea_rope_params_t* rope, int head_dim) {
+  if (!rope) return;
+  rope->axes_dim[0] = head_dim / 4;
+  rope->axes_dim[1] = 3 * head_dim / 8;
+  rope->axes_dim[2] = 3 * head_dim / 8;
+  rope->theta = 10000.0f;
+  rope->eps = 1e-6f;
+}
+
+namespace {
+int check_rope(const krea_rope_params_t* r, int head_dim) {
+  if (!r || !(r->theta > 0.f) || !(r->eps >= 0.f)) return KREA_ERR_INVALID_ARG;
+  int sum = 0;
+  for (int a = 0; a < 3; ++a) {
+    if (r->axes_dim[a] < 0 || r->axes_dim[a] % 2 != 0) return KREA_ERR_INVALID_ARG;
+    sum += r->axes_dim[a];
+  }
+  if (sum % 4 != 0 || (head_dim > 0 && sum > head_dim)) return KREA_ERR_INVALID_ARG;
+  return KREA_OK;
+}
+}  // namespace
+
+int krea_attn_rope_table(const int32_t* pos, int tokens, const krea_rope_params_t* rope, float* table,
+                         void* stream) {
+  int rc = check_rope(rope, 0);
+  if (rc != KREA_OK) return rc;
+  if (!pos || !table || tokens <= 0 || !aligned16(table) || (reinterpret_cast<uintptr_t>(pos) & 3)) return KREA_ERR_INVALID_ARG;
+  rc = check_device();
+  if (rc != KREA_OK) return rc;
+  return launch_rope_table(pos, tokens, rope->axes_dim, (double)rope->theta, table, stream);
+}
+
+int krea_attn_qk_prologue(const void* x, void* y, const float* gamma, const float* table, int batch, int tokens,
+                          int heads, int head_dim, int dtype, const int64_t* x_stride, const int64_t* y_stride,
+                          const krea_rope_params_t* rope, int8_t* codes, float* scales, void* stream) {
+  if (head_dim != 64 && head_dim != 128) return KREA_ERR_UNSUPPORTED;
+  if (dtype != KREA_F16 && dtype != KREA_BF16) return KREA_ERR_UNSUPPORTED;
+  int rc = check_rope(rope, head_dim);
+  if (rc != KREA_OK) return rc;
+  if (batch <= 0 || tokens <= 0 || heads <= 0 || batch > 65535 || heads > 65535 || !x || !y || !table ||
+      !x_stride || !y_stride)
+    return KREA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(table) || (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3)))
+    return KREA_ERR_INVALID_ARG;
+  if (!stride_ok(x_stride, 2) || !stride_ok(y_stride, 2)) return KREA_ERR_INVALID_ARG;
+  if (codes && (!scales || !aligned16(codes))) return KREA_ERR_INVALID_ARG;
+  rc = check_device();
+  if (rc != KREA_OK) return rc;
+  PrologueDevParams p;
+  p.x = x;
+  p.y = y;
+  p.gamma = gamma;
+  p.table = table;
+  p.codes = codes;
+  p.scales = scales;
+  for (int i = 0; i < 3; ++i) {
+    p.x_stride[i] = x_stride[i];
+    p.y_stride[i] = y_stride[i];
+  }
+  p.B = batch;
+  p.L = tokens;
+  p.H = heads;
+  p.d = head_dim;
+  p.nt = (tokens + kTile - 1) / kTile;
+  p.n_pairs = (rope->axes_dim[0] + rope->axes_dim[1] + rope->axes_dim[2]) / 2;
+  p.eps = rope->eps;
+  return launch_prologue(p, dtype == KREA_BF16, stream);
+}
+
 size_t krea_attn_workspace_bytes(int text_len, int grid_h, int grid_w, int mode,
                                  const krea_attn_params_t* p) {
   if (mode != KREA_MODE_TILEMIX || check_common(p) != KREA_OK) return 0;

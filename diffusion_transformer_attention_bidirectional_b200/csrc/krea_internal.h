@@ -49,6 +49,22 @@ int build_map(const Geometry& g, HostMap* out);
 int launch_build_map(const Geometry& g, int32_t* row_ptr, int32_t* packed, int32_t* col, uint8_t* kind,
                      int capacity, int32_t* status, void* stream);
 
+// QK prologue (prologue.cu): rotary table, then RMSNorm + rotation (+ INT8 codes).
+struct PrologueDevParams {
+  const void* x;
+  void* y;
+  const float* gamma;   // [d] or null (ones)
+  const float* table;   // [L][n_pairs][2] cos, sin
+  int8_t* codes;        // [B, L, H, d] or null
+  float* scales;        // [B, H, nt]
+  long long x_stride[3];
+  long long y_stride[3];
+  int B, L, H, d, nt, n_pairs;
+  float eps;
+};
+int launch_rope_table(const int32_t* pos, int tokens, const int axes[3], double theta, float* table, void* stream);
+int launch_prologue(const PrologueDevParams& p, bool bf16, void* stream);
+
 // Resolves and validates the geometry of a call.
 int make_geometry(int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* p,
                   Geometry* g);

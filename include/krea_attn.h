@@ -172,6 +172,47 @@ KREA_API int krea_attn_build_map_device(int text_len, int grid_h, int grid_w, in
                                         const krea_attn_params_t* params, int32_t* row_ptr, int32_t* col,
                                         uint8_t* kind, int32_t capacity, void* stream);
 
+/* QK prologue: RMSNorm, then the 3-axis rotary embedding -- the two steps the
+ * pages keep stock on q and k right before the attention core ("Krea 2 TileMix
+ * Attention (FP16/INT8 tiles)", section "What it actually patches"; the pages give
+ * no formula: the readings below are this library's), in one pass over HBM:
+ *   y = rope(x * gamma / sqrt(mean(x^2) + eps))   per (batch, token, head) vector.
+ * rope turns adjacent channel pairs (2i, 2i+1) of three consecutive channel
+ * groups of axes_dim[0], axes_dim[1], axes_dim[2] channels (text index, image row,
+ * image column; the channels after them pass unchanged) by
+ * pos[t][a] * theta^(-2i / axes_dim[a]) radians. */
+typedef struct {
+  int32_t axes_dim[3]; /* even; sum <= head_dim and a multiple of 4 */
+  float theta;         /* > 0 */
+  float eps;           /* >= 0, added to the mean square */
+} krea_rope_params_t;
+
+/* (head_dim/4, 3 head_dim/8, 3 head_dim/8) channels, theta 10000, eps 1e-6. */
+KREA_API void krea_attn_default_rope(krea_rope_params_t* rope, int head_dim);
+
+/* Rotary table of a geometry: table[t][j] = (cos, sin) of pair j's angle for
+ * token t (pairs numbered axis by axis), from pos [tokens][3] int32 (device),
+ * angles and trigonometry in fp64, stored as fp32 in table
+ * [tokens][n_pairs][2] (device, 16-byte aligned, n_pairs = sum(axes_dim) / 2).
+ * Build it once per geometry: every block and both q and k reuse it. */
+KREA_API int krea_attn_rope_table(const int32_t* pos, int tokens, const krea_rope_params_t* rope, float* table,
+                                  void* stream);
+
+/* y = rope(rmsnorm(x)) on device tensors x, y [batch, tokens, heads, head_dim]
+ * (element strides x_stride / y_stride over (batch, token, head), head_dim
+ * contiguous, rows 16-byte aligned; y may be x: in place). dtype KREA_F16 or
+ * KREA_BF16 for both; computed in fp32, rounded once. gamma: head_dim fp32
+ * weights (device) or NULL for ones. table: from krea_attn_rope_table with the
+ * same rope params. head_dim 64 or 128.
+ * If codes is not NULL, the pass also writes the TileMix INT8 codes of the stored
+ * y, codes [batch, tokens, heads, head_dim] contiguous, and scales [batch, heads,
+ * ceil(tokens / 128)] (one per 128-token block: absmax / 127), decided exactly as
+ * krea_attn_quantize decides them for queries. */
+KREA_API int krea_attn_qk_prologue(const void* x, void* y, const float* gamma, const float* table, int batch,
+                                   int tokens, int heads, int head_dim, int dtype, const int64_t* x_stride,
+                                   const int64_t* y_stride, const krea_rope_params_t* rope, int8_t* codes,
+                                   float* scales, void* stream);
+
 /* Run only the TileMix quantiser (key mean, centred keys, INT8 codes and scales)
  * into params->workspace, laid out as krea_attn_workspace_layout() says. */
 KREA_API int krea_attn_quantize(const void* q, const void* k, int text_len, int grid_h, int grid_w,

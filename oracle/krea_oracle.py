@@ -40,6 +40,17 @@ Readings taken where the pages are silent (each is listed in the design notes):
   centred, K centred by its per-(batch, kv head, channel) mean over all tokens
   when smooth_k; the centred K is used by the FP16 tiles too.
 
+QK prologue ([TM] "What it actually patches": QK RMSNorm and 3-axis RoPE are the
+steps right before the attention core; the pages name them and give no formula).
+Readings, each listed in the design notes: RMSNorm y = x * gamma / sqrt(mean(x^2)
++ eps) per (token, head) vector, gamma one weight per channel shared by the
+heads, eps 1e-6; then a rotary embedding over three consecutive channel groups
+of axes_dim channels (default d/4, 3d/8, 3d/8 = 32, 48, 48 at d = 128), adjacent
+channel pairs (2i, 2i+1) of group a turned by pos_a * theta^(-2i / axes_dim[a]),
+theta = 10000; positions: text token t at (t, 0, 0), image token at grid (r, c)
+at (0, r, c). Parity of this step is pinned by the closed forms and the
+rotation identities in the tests.
+
 Parity note: the INT8 quantisation scheme is fixed by the specification, not by
 the pages, so the INT8 path is pinned only by its error bound and by the pages'
 invariants (pattern zero equals dense, smooth_k leaves FP16 results unchanged).
@@ -393,6 +404,65 @@ def attention(case, q, k, v, gate=None, rows: Optional[Sequence[int]] = None,
     if return_probs:
         res["probs"] = probs
     return res
+
+
+# ----------------------------------------------------------------------------
+# QK prologue: RMSNorm, then the 3-axis rotary embedding
+# ----------------------------------------------------------------------------
+
+def default_axes(head_dim: int):
+    """Channel groups of the three rotary axes: d/4, 3d/8, 3d/8."""
+    return (head_dim // 4, 3 * head_dim // 8, 3 * head_dim // 8)
+
+
+def rope_positions(text_len: int, grid_h: int, grid_w: int) -> np.ndarray:
+    """[L, 3] positions: text token t at (t, 0, 0); image token (r, c) at (0, r, c)."""
+    L = text_len + grid_h * grid_w
+    pos = np.zeros((L, 3), dtype=np.int64)
+    pos[:text_len, 0] = np.arange(text_len)
+    for i in range(grid_h * grid_w):
+        pos[text_len + i, 1] = i // grid_w
+        pos[text_len + i, 2] = i % grid_w
+    return pos
+
+
+def rope_angles(pos: np.ndarray, axes_dim, theta: float = 10000.0) -> np.ndarray:
+    """[L, sum(axes_dim) / 2] rotation angles, pair by pair, axis by axis."""
+    cols = []
+    for a, n in enumerate(axes_dim):
+        for i in range(n // 2):
+            cols.append(pos[:, a].astype(np.float64) * theta ** (-2.0 * i / n))
+    return np.stack(cols, axis=1) if cols else np.zeros((pos.shape[0], 0))
+
+
+def rms_norm(x: np.ndarray, gamma: Optional[np.ndarray] = None, eps: float = 1e-6) -> np.ndarray:
+    """x [..., d] -> x * gamma / sqrt(mean over d of x^2 + eps), in fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    r = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    y = x / r
+    return y if gamma is None else y * np.asarray(gamma, dtype=np.float64)
+
+
+def rope_rotate(x: np.ndarray, ang: np.ndarray) -> np.ndarray:
+    """x [B, L, H, d]; ang [L, n] turns channel pairs (2j, 2j+1), j < n; the rest pass."""
+    x = np.array(x, dtype=np.float64)
+    n = ang.shape[1]
+    c = np.cos(ang)[None, :, None, :]
+    s = np.sin(ang)[None, :, None, :]
+    x0 = x[..., 0:2 * n:2].copy()
+    x1 = x[..., 1:2 * n:2].copy()
+    x[..., 0:2 * n:2] = x0 * c - x1 * s
+    x[..., 1:2 * n:2] = x0 * s + x1 * c
+    return x
+
+
+def qk_prologue(x, pos: np.ndarray, gamma: Optional[np.ndarray] = None, axes_dim=None,
+                theta: float = 10000.0, eps: float = 1e-6) -> np.ndarray:
+    """rope(rms_norm(x)) for x [B, L, H, d] (torch or numpy), in fp64."""
+    x = _as_f64(x)
+    d = x.shape[-1]
+    axes = default_axes(d) if axes_dim is None else tuple(axes_dim)
+    return rope_rotate(rms_norm(x, gamma, eps), rope_angles(pos, axes, theta))
 
 
 def admitted_pairs(case) -> int:

@@ -13,14 +13,15 @@ Shapes follow the Krea 2 renders the pages describe:
   section "What the mask actually is"); a 4 MP render a 128 x 128 grid (~16k tokens).
 * text prefix padded to 512 in training (same page, same section).
 
-Inputs for the attention core are post-RMSNorm / post-RoPE q, k and v in the
-layout [batch, tokens, heads, head_dim] (head_dim contiguous), plus the optional
-sigmoid-gate logits [batch, tokens, q_heads, head_dim].
+Tensors are q, k and v in the layout [batch, tokens, heads, head_dim] (head_dim
+contiguous), plus the optional sigmoid-gate logits [batch, tokens, q_heads,
+head_dim]. A case with `prologue=True` describes raw q/k projections: the q and
+k the attention sees are those after the QK prologue (RMSNorm + 3-axis RoPE),
+which is part of the method and is applied by whoever consumes the draws (the
+oracle in the tests, the library's prologue kernel on the GPU), never here.
 
 Random numbers come from numpy's PCG64 generator, one independent stream per
-(seed, tensor) pair, drawn in float32 and rounded once to the storage dtype
-(the RMS-normalised, rotated q/k of the 1 MP dense case are computed in fp64
-from those draws before the rounding).
+(seed, tensor) pair, drawn in float32 and rounded once to the storage dtype.
 """
 from __future__ import annotations
 
@@ -54,7 +55,8 @@ class Case:
     mode: str = "dense"            # "dense" | "tilemix" | "scanline"
     seed: int = 0
     gate: bool = False
-    qk_dist: str = "normal"        # "normal" | "rms_rope" | "normal_koffset"
+    qk_dist: str = "normal"        # "normal" | "normal_koffset"
+    prologue: bool = False         # q/k are raw projections: the QK prologue comes first
     softmax_scale: float = 0.0     # 0 -> 1/sqrt(head_dim)
     # TileMix
     pattern: str = "band"          # "zero" | "band" | "one"
@@ -84,55 +86,13 @@ def _normal(seed: int, stream: str, shape, mean: float = 0.0, std: float = 1.0) 
     return x
 
 
-def _rope_angles(case: Case) -> np.ndarray:
-    """Angles [L, head_dim/2] of a 3-axis rotary embedding (generator choice only).
-
-    Axis split (32, 48, 48) channels, base 10000, adjacent-pair rotation. Text
-    token t sits at (t, 0, 0); image token at grid (r, c) sits at (0, r, c).
-    The pages only name "3-axis RoPE"; any fixed choice gives inputs of the
-    right structure, and nothing downstream depends on which one.
-    """
-    d = case.head_dim
-    dims = (d // 4, 3 * d // 8, 3 * d // 8)
-    T, H, W = case.text_len, case.grid_h, case.grid_w
-    L = T + H * W
-    pos = np.zeros((L, 3), dtype=np.float64)
-    pos[:T, 0] = np.arange(T)
-    rr, cc = np.meshgrid(np.arange(H), np.arange(W), indexing="ij")
-    pos[T:, 1] = rr.reshape(-1)
-    pos[T:, 2] = cc.reshape(-1)
-    parts = []
-    for axis, n in enumerate(dims):
-        inv = 10000.0 ** (-np.arange(0, n, 2, dtype=np.float64) / n)
-        parts.append(pos[:, axis : axis + 1] * inv[None, :])
-    return np.concatenate(parts, axis=1)
-
-
-def _rms_rope(x: np.ndarray, ang: np.ndarray) -> np.ndarray:
-    """Per-(token, head) RMS normalisation, then pairwise rotation by `ang`."""
-    rms = np.sqrt(np.mean(x * x, axis=-1, keepdims=True))
-    x = x / rms
-    c = np.cos(ang)[None, :, None, :]
-    s = np.sin(ang)[None, :, None, :]
-    x0 = x[..., 0::2]
-    x1 = x[..., 1::2]
-    y = np.empty_like(x)
-    y[..., 0::2] = x0 * c - x1 * s
-    y[..., 1::2] = x0 * s + x1 * c
-    return y
-
-
 def make_inputs(case: Case, with_gate: Optional[bool] = None):
     """Return CPU torch tensors (q, k, v, gate-or-None) in the case's dtype."""
     B, L, Hq, Hkv, d = case.batch, case.seq_len, case.q_heads, case.kv_heads, case.head_dim
     q = _normal(case.seed, "q", (B, L, Hq, d))
     k = _normal(case.seed, "k", (B, L, Hkv, d))
     v = _normal(case.seed, "v", (B, L, Hkv, d))
-    if case.qk_dist == "rms_rope":
-        ang = _rope_angles(case)
-        q = _rms_rope(q.astype(np.float64), ang)
-        k = _rms_rope(k.astype(np.float64), ang)
-    elif case.qk_dist == "normal_koffset":
+    if case.qk_dist == "normal_koffset":
         # a shared per-(kv head, channel) offset ~ N(0.5, 0.1) on every key
         off = _normal(case.seed, "koff", (1, 1, Hkv, d), mean=0.5, std=0.1)
         k = k + off
@@ -159,9 +119,10 @@ def tiny_dense() -> Case:
 
 
 def dense_1mp() -> Case:
-    """Krea 2 1 MP: 48/12 heads, d=128, 512 text + 64x64 grid, bf16 RMS+RoPE q/k, gate."""
+    """Krea 2 1 MP: 48/12 heads, d=128, 512 text + 64x64 grid, bf16, gate; q/k are raw
+    projections that go through the QK prologue (RMSNorm + 3-axis RoPE) first."""
     return Case("dense_1mp", 1, 48, 12, 128, 512, 64, 64, dtype="bf16", mode="dense", seed=2,
-                gate=True, qk_dist="rms_rope")
+                gate=True, prologue=True)
 
 
 def scanline_1mp() -> Case:

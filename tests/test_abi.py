@@ -107,3 +107,29 @@ def test_workspace_sizes():
     assert K.workspace_bytes("dense", 512, 128, 128, p) == 0
     for k in ("kc", "q8", "k8", "sq", "sk", "mu", "part"):
         assert lay[k] % 256 == 0
+
+
+def test_prologue_arguments_rejected_without_gpu():
+    L = _lib.lib()
+    r = K.rope_params(128)
+    assert tuple(r.axes_dim) == (32, 48, 48) and abs(r.theta - 1e4) < 1e-3 and abs(r.eps - 1e-6) < 1e-12
+    s = (ctypes.c_int64 * 3)(1 << 20, 1024, 128)
+    ptr = 1 << 20
+
+    def call(rope, d=128, dtype=1, x=ptr):
+        return L.krea_attn_qk_prologue(x, ptr, None, ptr, 1, 8, 8, d, dtype, s, s, ctypes.byref(rope), None, None,
+                                       None)
+
+    assert call(r, d=96) == _lib.ERR_UNSUPPORTED
+    assert call(r, dtype=2) == _lib.ERR_UNSUPPORTED          # fp32
+    assert call(r, x=ptr + 8) == _lib.ERR_INVALID_ARG         # misaligned rows
+    bad = K.rope_params(128, axes_dim=(32, 47, 49))           # odd axis
+    assert call(bad) == _lib.ERR_INVALID_ARG
+    big = K.rope_params(128, axes_dim=(64, 48, 48))           # more rotary channels than head_dim
+    assert call(big) == _lib.ERR_INVALID_ARG
+    assert L.krea_attn_rope_table(ptr, 8, ctypes.byref(K.rope_params(128, theta=-1.0)), ptr, None) == -1
+
+
+def test_rope_positions_layout():
+    pos = K.rope_positions(2, 2, 3)
+    assert pos.tolist() == [[0, 0, 0], [1, 0, 0], [0, 0, 0], [0, 0, 1], [0, 0, 2], [0, 1, 0], [0, 1, 1], [0, 1, 2]]

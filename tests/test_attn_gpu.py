@@ -175,6 +175,10 @@ def test_quantizer_matches_oracle_fp32_decisions():
 def test_config_dense_1mp():
     c = S.dense_1mp()
     q, k, v, g = S.make_inputs(c)
+    # raw projections through the oracle's QK prologue (RMSNorm + 3-axis RoPE), rounded to bf16
+    pos = ko.rope_positions(c.text_len, c.grid_h, c.grid_w)
+    q = torch.from_numpy(ko.qk_prologue(q, pos)).to(torch.bfloat16)
+    k = torch.from_numpy(ko.qk_prologue(k, pos)).to(torch.bfloat16)
     out = gpu_run(c, q, k, v, g)
     rows = tile_rows(c.seq_len, [0, 3, 4, 17, 35])
     # thousands of keys per row: the bf16 rounding of P averages out below 5e-4

@@ -364,3 +364,67 @@ def test_admitted_pair_counts_closed_form():
     assert ko.admitted_pairs(Case("s", 1, 1, 1, 128, T, H, W, mode="scanline", tile_aligned=True, **base)) == aligned
     # dense: every pair of real tokens
     assert ko.admitted_pairs(Case("d", 1, 1, 1, 128, T, H, W, mode="dense")) == L * L
+
+
+# ---------------------------------------------------------------------------- QK prologue pins
+
+def test_rms_norm_closed_forms():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((2, 5, 3, 128)) * 3.0
+    y = ko.rms_norm(x, eps=0.0)
+    assert np.allclose(np.mean(y * y, axis=-1), 1.0, atol=1e-13)     # unit RMS per vector
+    assert np.allclose(ko.rms_norm(7.5 * x, eps=0.0), y, atol=1e-13)  # scale invariance
+    g = rng.standard_normal(128)
+    assert np.allclose(ko.rms_norm(x, g, eps=0.0), y * g, atol=1e-13)  # one weight per channel
+    # eps enters under the root: mean(y^2) = m / (m + eps), m = mean(x^2)
+    m = np.mean(x * x, axis=-1)
+    ye = ko.rms_norm(x, eps=0.5)
+    assert np.allclose(np.mean(ye * ye, axis=-1), m / (m + 0.5), atol=1e-13)
+
+
+def test_rope_positions_layout():
+    pos = ko.rope_positions(2, 2, 3)
+    assert pos.tolist() == [[0, 0, 0], [1, 0, 0], [0, 0, 0], [0, 0, 1], [0, 0, 2], [0, 1, 0], [0, 1, 1], [0, 1, 2]]
+    assert ko.default_axes(128) == (32, 48, 48) and ko.default_axes(64) == (16, 24, 24)
+
+
+def test_rope_worked_example_and_frequencies():
+    # d = 4, axes (2, 2, 0): pair 0 turns by p0 * theta^0, pair 1 by p1 * theta^0
+    x = np.array([1.0, 0.0, 1.0, 0.0]).reshape(1, 1, 1, 4)
+    pos = np.array([[1, 2, 0]])
+    y = ko.rope_rotate(x, ko.rope_angles(pos, (2, 2, 0)))[0, 0, 0]
+    assert np.allclose(y, [math.cos(1), math.sin(1), math.cos(2), math.sin(2)], atol=1e-15)
+    # pair i of an axis of n channels turns at theta^(-2i/n) radians per position step
+    ang = ko.rope_angles(np.array([[0, 1, 0]]), (32, 48, 48))[0]
+    assert np.all(ang[:16] == 0) and np.all(ang[40:] == 0)
+    assert np.allclose(ang[16:40], [10000.0 ** (-2.0 * i / 48) for i in range(24)], rtol=1e-15)
+
+
+def test_rope_rotation_identities():
+    rng = np.random.default_rng(5)
+    L, d = 6, 128
+    axes = ko.default_axes(d)
+    q = rng.standard_normal((1, L, 1, d))
+    k = rng.standard_normal((1, L, 1, d))
+    p1 = rng.integers(0, 50, size=(L, 3))
+    p2 = rng.integers(0, 50, size=(L, 3))
+    r = lambda x, p: ko.rope_rotate(x, ko.rope_angles(p, axes))
+    assert np.allclose(r(q, np.zeros((L, 3), dtype=np.int64)), q, atol=0)           # position 0: identity
+    pair = lambda x: x[..., 0::2] ** 2 + x[..., 1::2] ** 2
+    assert np.allclose(pair(r(q, p1)), pair(q), atol=1e-12)                          # a rotation per pair
+    assert np.allclose(r(r(q, p1), p2), r(q, p1 + p2), atol=1e-11)                   # angles add
+    # relative position: <R(a) q, R(b) k> = <R(a - b) q, k>
+    lhs = np.sum(r(q, p1) * r(k, p2), axis=-1)
+    rhs = np.sum(r(q, p1 - p2) * k, axis=-1)
+    assert np.allclose(lhs, rhs, atol=1e-11)
+
+
+def test_qk_prologue_is_norm_then_rope():
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((1, 12, 2, 64))
+    pos = ko.rope_positions(4, 2, 4)
+    g = rng.uniform(0.5, 1.5, 64)
+    y = ko.qk_prologue(x, pos, g)
+    # rotation keeps each pair's length, so the RMS of y is that of the normalised x
+    assert np.allclose(np.mean(y * y, -1), np.mean(ko.rms_norm(x, g) ** 2, -1), atol=1e-12)
+    assert np.allclose(y[:, 0], ko.rms_norm(x, g)[:, 0], atol=0)  # token 0 sits at (0, 0, 0)
