@@ -205,6 +205,35 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- our arm
+def time_prologue(K, device, stream, flush, P, reps: int = 8):
+    """The QK prologue (RMSNorm + 3-axis RoPE, one HBM pass) at the 4 MP shape, bound
+    by HBM: algorithmic bytes = every q and k row read once and written once."""
+    from synth import inputs as S
+
+    pc = S.Case("prologue_4mp", 1, 48, 12, 128, 512, 128, 128, dtype="bf16", mode="dense", seed=91, prologue=True)
+    q_raw, k_raw, _, _ = S.make_inputs(pc)
+    qd, kd = q_raw.to(device), k_raw.to(device)
+    qo, ko_ = torch.empty_like(qd), torch.empty_like(kd)
+    table = K.rope_table(K.rope_positions(pc.text_len, pc.grid_h, pc.grid_w, device))
+    times = []
+    for it in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        K.qk_prologue(qd, table, out=qo)
+        K.qk_prologue(kd, table, out=ko_)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        if it >= 3:
+            times.append(a.elapsed_time(b))
+    ms = sorted(times)[len(times) // 2]
+    nbytes = 2 * (qd.numel() + kd.numel()) * qd.element_size()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": "prologue_kernel<bf16, 128> (q then k)", "ms": round(ms, 4), "algorithmic_bytes": nbytes,
+            "achieved_gbs": round(gbs, 1), "peak_gbs": P["hbm_gbs"], "frac": round(gbs / P["hbm_gbs"], 4),
+            "bound": "hbm", "peak_source": f"{P['source']} copy bandwidth", "l2": "flushed before each pass"}
+
+
 def run_ours(args, rank, world, device):
     import diffusion_transformer_attention_bidirectional_b200 as K
     from synth import inputs as S
@@ -354,6 +383,8 @@ def run_ours(args, rank, world, device):
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during the comparisons")
 
+    prologue = None if args.no_comparisons else time_prologue(K, device, stream, flush, P)
+
     # roofline of the dominant kernel: the attention kernel on the dense variant
     # (its launches are attention kernels only), algorithmic FLOPs / event time
     dense_attn_ms = attn_dense_ms / args.steps
@@ -398,6 +429,8 @@ def run_ours(args, rank, world, device):
         "variants": variants,
         "comparisons": comparisons,
     }
+    if prologue is not None:
+        res["prologue"] = prologue
     dense_tf = next((v["tflops"] for n, v in variants.items() if "cfg_pair" in n), None)
     for n, v in variants.items():
         if dense_tf and n.startswith("scanline"):
@@ -477,6 +510,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prologue-only", action="store_true",
+                    help="time only the QK prologue at the 4 MP shape (profiling)")
     ap.add_argument("--no-comparisons", action="store_true",
                     help="skip the band-vs-zero timing after the timed steps (launch-list captures)")
     ap.add_argument("--case", default=None,
@@ -503,6 +538,13 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
+    if args.prologue_only:
+        import diffusion_transformer_attention_bidirectional_b200 as K
+
+        torch.cuda.set_device(device)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        print(json.dumps(time_prologue(K, device, torch.cuda.current_stream(device), flush, peaks())), flush=True)
+        return
     try:
         res = run_ours(args, rank, world, device)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -58,86 +58,113 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const int32_t* pos, int
   table[idx] = make_float2((float)c, (float)s);
 }
 
-// Grid (ceil(L / 128), H, B), 128 threads: thread = token, its whole row in registers.
-template <bool BF16, int D>
-__global__ void __launch_bounds__(128) prologue_kernel(PrologueDevParams p) {
+// Grid (ceil(L / 128), H, B), 512 threads = 16 warps x 8 rows of the CTA's
+// 128-token block. A row of d channels is held by d/8 lanes, 8 channels (16
+// bytes) each, so one warp access covers 32 / (d/8) whole rows: 512 contiguous
+// bytes per row pair at d = 128. Channel pairs (2i, 2i+1) never straddle lanes.
+template <bool BF16, int D, bool CODES>
+__global__ void __launch_bounds__(512, CODES ? 1 : 2) prologue_kernel(PrologueDevParams p) {
+  constexpr int LPR = D / 8;       // lanes per row
+  constexpr int RPW = 32 / LPR;    // rows per warp access
+  constexpr int STEPS = 8 / RPW;   // accesses per warp for its 8 rows
   const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int t = blk * kTile + threadIdx.x;
-  const bool live = t < p.L;
-  __shared__ float red[4];
-  float x[D];
-  float amax = 0.f;
-  if (live) {
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + b * p.x_stride[0] +
-                                                      (long long)t * p.x_stride[1] + h * p.x_stride[2]);
-    float ss = 0.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane / LPR, li = lane % LPR;
+  const int c0 = 8 * li;            // this lane's channels c0 .. c0 + 7
+  const int pj0 = c0 / 2;           // and its rotary pairs pj0 .. pj0 + 3
+  __shared__ float red[16];
+  float g[8];
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      const uint4 u = src[i];
+  for (int j = 0; j < 8; ++j) g[j] = p.gamma ? p.gamma[c0 + j] : 1.0f;
+  float keep[CODES ? STEPS : 1][8];  // stored values, for the codes
+  float amax = 0.f;
+  uint4 raw[STEPS];  // every load of the thread is issued before the first use
+#pragma unroll
+  for (int st = 0; st < STEPS; ++st) {
+    const int t = blk * kTile + warp * 8 + st * RPW + sub;
+    raw[st] = t < p.L ? *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + b * p.x_stride[0] +
+                                                        (long long)t * p.x_stride[1] + h * p.x_stride[2] + c0)
+                      : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int st = 0; st < STEPS; ++st) {
+    const int t = blk * kTile + warp * 8 + st * RPW + sub;
+    const bool live = t < p.L;
+    float x[8];
+    float ss = 0.f;
+    if (live) {
+      const uint4 u = raw[st];
       const uint16_t* e = reinterpret_cast<const uint16_t*>(&u);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        x[8 * i + j] = ld_f<BF16>(e[j]);
-        ss = __fmaf_rn(x[8 * i + j], x[8 * i + j], ss);
+        x[j] = ld_f<BF16>(e[j]);
+        ss = __fmaf_rn(x[j], x[j], ss);
       }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[j] = 0.f;
     }
-    // 1 / sqrt(mean + eps), each step rounded once (IEEE)
-    const float r = __frsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)D), p.eps));
 #pragma unroll
-    for (int c = 0; c < D; ++c) x[c] = p.gamma ? __fmul_rn(__fmul_rn(x[c], r), p.gamma[c]) : __fmul_rn(x[c], r);
-    const float4* tab = reinterpret_cast<const float4*>(p.table + 2LL * t * p.n_pairs);  // (cos, sin) pairs
+    for (int o = LPR / 2; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+    if (live) {
+      // 1 / sqrt(mean + eps), each step rounded once (IEEE)
+      const float r = __frsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)D), p.eps));
 #pragma unroll
-    for (int j2 = 0; j2 < D / 4; ++j2) {  // two pairs per 16-byte table load
-      if (2 * j2 >= p.n_pairs) break;
-      const float4 cs = tab[j2];
-      const float c0 = cs.x, s0 = cs.y, c1 = cs.z, s1 = cs.w;
-      const float a0 = x[4 * j2], a1 = x[4 * j2 + 1];
-      x[4 * j2] = __fmaf_rn(a0, c0, -__fmul_rn(a1, s0));
-      x[4 * j2 + 1] = __fmaf_rn(a0, s0, __fmul_rn(a1, c0));
-      if (2 * j2 + 1 < p.n_pairs) {
-        const float b0 = x[4 * j2 + 2], b1 = x[4 * j2 + 3];
-        x[4 * j2 + 2] = __fmaf_rn(b0, c1, -__fmul_rn(b1, s1));
-        x[4 * j2 + 3] = __fmaf_rn(b0, s1, __fmul_rn(b1, c1));
+      for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(__fmul_rn(x[j], r), g[j]);
+      const float4* tab = reinterpret_cast<const float4*>(p.table + 2LL * ((long long)t * p.n_pairs + pj0));
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {  // two pairs per 16-byte table load
+        if (pj0 + 2 * q2 >= p.n_pairs) break;
+        const float4 cs = tab[q2];
+        const float a0 = x[4 * q2], a1 = x[4 * q2 + 1], b0 = x[4 * q2 + 2], b1 = x[4 * q2 + 3];
+        x[4 * q2] = __fmaf_rn(a0, cs.x, -__fmul_rn(a1, cs.y));
+        x[4 * q2 + 1] = __fmaf_rn(a0, cs.y, __fmul_rn(a1, cs.x));
+        x[4 * q2 + 2] = __fmaf_rn(b0, cs.z, -__fmul_rn(b1, cs.w));
+        x[4 * q2 + 3] = __fmaf_rn(b0, cs.w, __fmul_rn(b1, cs.z));
       }
-    }
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.y) + b * p.y_stride[0] +
-                                          (long long)t * p.y_stride[1] + h * p.y_stride[2]);
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
       uint4 u;
       uint16_t* e = reinterpret_cast<uint16_t*>(&u);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        e[j] = st_f<BF16>(x[8 * i + j]);
-        x[8 * i + j] = ld_f<BF16>(e[j]);  // the codes below are decided on the stored values
-        amax = fmaxf(amax, fabsf(x[8 * i + j]));
+        e[j] = st_f<BF16>(x[j]);
+        if constexpr (CODES) {
+          keep[st][j] = ld_f<BF16>(e[j]);  // the codes below are decided on the stored values
+          amax = fmaxf(amax, fabsf(keep[st][j]));
+        }
       }
-      dst[i] = u;
+      *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.y) + b * p.y_stride[0] + (long long)t * p.y_stride[1] +
+                                h * p.y_stride[2] + c0) = u;
+    } else if constexpr (CODES) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) keep[st][j] = 0.f;
     }
   }
-  if (!p.codes) return;  // uniform over the grid
+  if constexpr (!CODES) return;
+  else {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  if (lane == 0) red[warp] = amax;
   __syncthreads();
-  amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  amax = red[0];
+#pragma unroll
+  for (int w = 1; w < 16; ++w) amax = fmaxf(amax, red[w]);
   const float scale = __fdiv_rn(amax, 127.0f);
   const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
   if (threadIdx.x == 0) p.scales[((long long)b * p.H + h) * p.nt + blk] = scale;
-  if (live) {
-    int8_t* dst8 = p.codes + (((long long)b * p.L + t) * p.H + h) * D;
 #pragma unroll
-    for (int i = 0; i < D / 16; ++i) {
-      uint4 u;
-      int8_t* e = reinterpret_cast<int8_t*>(&u);
+  for (int st = 0; st < STEPS; ++st) {
+    const int t = blk * kTile + warp * 8 + st * RPW + sub;
+    if (t >= p.L) continue;
+    uint2 u;
+    int8_t* e = reinterpret_cast<int8_t*>(&u);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        float q = rintf(__fmul_rn(x[16 * i + j], inv));
-        q = fminf(fmaxf(q, -127.f), 127.f);
-        e[j] = (int8_t)(int)q;
-      }
-      reinterpret_cast<uint4*>(dst8)[i] = u;
+    for (int j = 0; j < 8; ++j) {
+      float q = rintf(__fmul_rn(keep[st][j], inv));
+      q = fminf(fmaxf(q, -127.f), 127.f);
+      e[j] = (int8_t)(int)q;
     }
+    *reinterpret_cast<uint2*>(p.codes + (((long long)b * p.L + t) * p.H + h) * D + c0) = u;
+  }
   }
 }
 
@@ -155,12 +182,17 @@ int launch_rope_table(const int32_t* pos, int tokens, const int axes[3], double 
 int launch_prologue(const PrologueDevParams& p, bool bf16, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const dim3 grid((unsigned)p.nt, (unsigned)p.H, (unsigned)p.B);
+  const bool codes = p.codes != nullptr;
   if (p.d == 128) {
-    if (bf16) prologue_kernel<true, 128><<<grid, 128, 0, s>>>(p);
-    else prologue_kernel<false, 128><<<grid, 128, 0, s>>>(p);
+    if (bf16) codes ? prologue_kernel<true, 128, true><<<grid, 512, 0, s>>>(p)
+                    : prologue_kernel<true, 128, false><<<grid, 512, 0, s>>>(p);
+    else codes ? prologue_kernel<false, 128, true><<<grid, 512, 0, s>>>(p)
+               : prologue_kernel<false, 128, false><<<grid, 512, 0, s>>>(p);
   } else if (p.d == 64) {
-    if (bf16) prologue_kernel<true, 64><<<grid, 128, 0, s>>>(p);
-    else prologue_kernel<false, 64><<<grid, 128, 0, s>>>(p);
+    if (bf16) codes ? prologue_kernel<true, 64, true><<<grid, 512, 0, s>>>(p)
+                    : prologue_kernel<true, 64, false><<<grid, 512, 0, s>>>(p);
+    else codes ? prologue_kernel<false, 64, true><<<grid, 512, 0, s>>>(p)
+               : prologue_kernel<false, 64, false><<<grid, 512, 0, s>>>(p);
   } else {
     return KREA_ERR_UNSUPPORTED;
   }
