@@ -97,7 +97,13 @@ def admitted_pairs(case, K) -> int:
     L = case.seq_len
     if case.mode != "scanline":
         return L * L
-    assert case.tile_aligned
+    T, H, W = case.text_len, case.grid_h, case.grid_w
+    if not case.tile_aligned:
+        # token rule: text queries see all L keys, image queries the T text keys and
+        # the W keys of every row within window // 2 of their own
+        half = case.window // 2
+        rows = sum(min(H - 1, r + half) - max(0, r - half) + 1 for r in range(H))
+        return T * L + H * W * T + rows * W * W
     rp, col, _ = K.get_map("scanline", case.text_len, case.grid_h, case.grid_w, window=case.window,
                            tile_aligned=True, text_pad=case.text_pad)
     T, N = case.text_len, case.grid_h * case.grid_w
@@ -380,6 +386,35 @@ def run_ours(args, rank, world, device):
             "band_ms": round(med["band"], 4), "zero_ms": round(med["zero"], 4),
             "speedup": round(med["zero"] / med["band"], 4),
             "modelled_speedup": round(2 * len(kind) / (2 * (len(kind) - n8) + 1.5 * n8), 4)}
+    # Scanline token rule (tile_aligned off) against tile-aligned at 1 MP, where the
+    # 64-token rows put two rows in a tile and the two rules differ.
+    if not args.no_comparisons:
+        from synth import inputs as S
+
+        base = S.scanline_1mp()
+        q1, k1, v1, _ = (t.to(device) if t is not None else None for t in S.make_inputs(base))
+        o1 = torch.empty(q1.shape, dtype=torch.float32, device=device)
+        rec = {}
+        for name, ta in (("tile_aligned", True), ("token_rule", False)):
+            c = dataclasses.replace(base, tile_aligned=ta)
+            fns, _ = make_call(c, K, (q1, k1, v1, None, o1), None, status)
+            times = []
+            for it in range(8):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for fn in fns:
+                    fn()
+                b.record(stream)
+                torch.cuda.synchronize(device)
+                if it >= 3:
+                    times.append(a.elapsed_time(b))
+            ms = sorted(times)[len(times) // 2]
+            pairs = admitted_pairs(c, K)
+            rec[name] = {"ms": round(ms, 4), "admitted_pairs": pairs,
+                         "tflops": round(case_flops(c, K) / (ms * 1e-3) / 1e12, 1)}
+        comparisons["scanline_1mp_token_rule_vs_tile_aligned"] = rec
+        del q1, k1, v1, o1
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during the comparisons")
 
