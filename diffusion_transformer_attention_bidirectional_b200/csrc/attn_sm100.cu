@@ -29,7 +29,9 @@
 // TMEM (512 columns x 128 lanes): S0 [0,128) S1 [128,256) O0 [256,384)
 // O1 [384,512); P_i (16-bit, 64 columns) overwrites the first half of S_i.
 // Per kv tile j and head i the MMA thread issues, in order,
-//   PV_i(j-1): O_i += P_i V_{j-1}   then   QK_i(j): S_i = Q_i K_j^T
+//   PV_i(j-1) on keys 0..63 (as soon as the softmax has written that half of
+//   P_i), PV_i(j-1) on keys 64..127 (when all of P_i is written), then
+//   QK_i(j): S_i = Q_i K_j^T
 // and commits S_i after QK_i(j); tcgen05 operations of one thread complete in
 // issue order, so when softmax i sees S_i(j) complete, PV_i(j-1) is complete
 // too and O_i may be rescaled in place before P_i(j) is released.
@@ -68,7 +70,8 @@ constexpr int BAR_Q = 0, BAR_FULL = 1, BAR_EMPTY = BAR_FULL + kSlots, BAR_S = BA
               BAR_GATE = BAR_QFREE + 1,   // gate tiles landed in the Q area
               BAR_EPI = BAR_GATE + 1,     // 2: all 128 rows of head i staged for the TMA store
               BAR_Q8 = BAR_EPI + 2,       // INT8 query codes landed (rows with INT8 tiles only)
-              N_BARS = BAR_Q8 + 1;
+              BAR_PH = BAR_Q8 + 1,        // 2: the first half of P_i (keys 0..63) written
+              N_BARS = BAR_PH + 2;
 constexpr uint32_t SM_TMEM_PTR = SM_BAR + 8 * N_BARS;
 constexpr uint32_t SM_ABORT = SM_TMEM_PTR + 4;
 constexpr uint32_t SMEM_USED = SM_BAR + 256;
@@ -207,11 +210,14 @@ __device__ __forceinline__ float i2f_exact(uint32_t x) {
 // v: the row of S (fp32 bits, or s32 for INT8 tiles), overwritten. mult: score
 // scale in log2 units (softmax scale * log2 e, times s_q s_k for INT8 tiles).
 // Key column c is admitted iff c < a1 or a2 <= c < a3 (masked tiles only).
-// Writes P (16-bit pairs) over the first 64 columns of S; updates m, l and,
-// when the running maximum moves, rescales O in TMEM.
+// Writes P (16-bit pairs) over the first 64 columns of S, releasing the first 32
+// (keys 0..63) on half_bar before the exponentials of keys 64..127 are taken, so
+// that PV on those keys overlaps them; updates m, l and, when the running maximum
+// moves, rescales O in TMEM (before either half of P is released).
 template <bool BF16, bool IS8, bool MASKED, bool ALL_POLY>
 __device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int a1, int a2, int a3, float& m,
-                                             float& l, bool first, uint32_t tS, uint32_t tO, int d) {
+                                             float& l, bool first, uint32_t tS, uint32_t tO, int d,
+                                             uint32_t half_bar) {
 #pragma unroll
   for (int c = 0; c < 128; ++c) {
     float r = IS8 ? i2f_exact(v[c]) : __uint_as_float(v[c]);
@@ -272,6 +278,12 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int
       pk[i] = pack2<BF16>(p0, p1);
     }
     ptx::tmem_st32(tS + 32u * h, pk);
+    if (h == 0) {  // keys 0..63 of P are in TMEM: the tensor core may start on them
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(half_bar);
+    }
   }
   float s0, s1, s2, s3;
   ptx::unf2(acc0, s0, s1);
@@ -315,13 +327,14 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
       }
     }
   };
-  auto pv = [&](int i, uint32_t slot, uint32_t acc) {
+  // PV over keys 64 half .. 64 half + 63 of the tile
+  auto pv = [&](int i, uint32_t slot, int half, uint32_t acc) {
     const uint32_t dO = tmem + 256u + (uint32_t)i * 128u;
-    const uint32_t aP = tmem + (uint32_t)i * 128u;
-    const uint32_t vd = dv + slot * (kTileBytes >> 4);
+    const uint32_t aP = tmem + (uint32_t)i * 128u + 32u * (uint32_t)half;
+    const uint32_t vd = dv + slot * (kTileBytes >> 4) + 512u * (uint32_t)half;  // 64 rows x 128 B
     ptx::mma_f16_ts_lo(dO, aP, vd, ID_PV, acc);
 #pragma unroll
-    for (int k = 1; k < 8; ++k)  // 16 keys per step: 8 TMEM columns of P, 16 rows of V (2 KB)
+    for (int k = 1; k < 4; ++k)  // 16 keys per step: 8 TMEM columns of P, 16 rows of V (2 KB)
       ptx::mma_f16_ts_lo(dO, aP + 8u * k, vd + 128u * k, ID_PV, 1);
   };
   bool ok = wait1(ctl, bar(BAR_Q), 0);
@@ -361,10 +374,14 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
       const int kind_next = e_next & 3;
       if (t + 2 < n) e_next = p.entries[e0 + t + 2];
       for (int i = 0; i < nh && ok; ++i) {
-        ok = wait1(ctl, bar(BAR_P + i), t & 1);
+        ok = wait1(ctl, bar(BAR_PH + i), t & 1);  // keys 0..63 of P_i(t)
         if (!ok) break;
         ptx::tc_fence_after();
-        pv(i, slot_v, t > 0 ? 1u : 0u);
+        pv(i, slot_v, 0, t > 0 ? 1u : 0u);
+        ok = wait1(ctl, bar(BAR_P + i), t & 1);   // all of P_i(t)
+        if (!ok) break;
+        ptx::tc_fence_after();
+        pv(i, slot_v, 1, 1u);
         if (has_next) {
           if (i == 0) {
             ok = wait1(ctl, bar(BAR_FULL + slot_k), (it / kSlots) & 1) && need_q8(kind_next);
@@ -450,6 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(bar(BAR_QFREE), 1);
     ptx::mbar_init(bar(BAR_GATE), 1);
     ptx::mbar_init(bar(BAR_Q8), 1);
+    ptx::mbar_init(bar(BAR_PH + 0), 4);  // one arrival per softmax warp
+    ptx::mbar_init(bar(BAR_PH + 1), 4);
     ptx::mbar_init(bar(BAR_EPI + 0), 128);
     ptx::mbar_init(bar(BAR_EPI + 1), 128);
     *abort_flag = 0;
@@ -601,10 +620,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s0 = kb * kTile;
         const int a1 = p.T - s0, a2 = klo - s0, a3 = khi - s0;
         const bool first = t == 0;
-        if (kind == 0) softmax_tile<BF16, false, false, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d);
-        else if (kind == 1) softmax_tile<BF16, false, true, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d);
-        else if (kind == 2) softmax_tile<BF16, true, false, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d);
-        else softmax_tile<BF16, true, true, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d);
+        if (kind == 0) softmax_tile<BF16, false, false, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, bar(BAR_PH + wg));
+        else if (kind == 1) softmax_tile<BF16, false, true, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, bar(BAR_PH + wg));
+        else if (kind == 2) softmax_tile<BF16, true, false, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, bar(BAR_PH + wg));
+        else softmax_tile<BF16, true, true, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, bar(BAR_PH + wg));
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
