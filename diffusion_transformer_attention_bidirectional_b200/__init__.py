@@ -188,14 +188,15 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[
               text_len: int, grid_h: int, grid_w: int, mode: str = "dense",
               out: Optional[torch.Tensor] = None, out_dtype: Optional[torch.dtype] = torch.float32,
               workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
-              stream: Optional[torch.cuda.Stream] = None, **opts) -> torch.Tensor:
+              stream: Optional[torch.cuda.Stream] = None, lse: Optional[torch.Tensor] = None,
+              **opts) -> torch.Tensor:
     """out = sigmoid(gate) * softmax(scale q k^T over the admitted keys) v, per query head.
 
     q [B, L, Hq, d], k and v [B, L, Hkv, d], gate [B, L, Hq, d] or None; L = text_len + grid_h * grid_w.
     mode: "dense" | "tilemix" | "scanline"; `opts` are make_params keywords (q_start, q_len,
     pattern, percentage, band_blocks, smooth_k, window, tile_aligned, text_pad, ...).
     """
-    _check_inputs(q, k, v, gate, out, workspace, status)
+    _check_inputs(q, k, v, gate, out, workspace, status, lse)
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     in_dt = _TORCH_DT[q.dtype]
@@ -216,6 +217,10 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         p.workspace = workspace.data_ptr()
         p.workspace_bytes = workspace.numel() * workspace.element_size()
+    if lse is not None:  # [B, Hq, L] fp32: ln sum_j exp(scale s_ij) per valid query row
+        if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, L):
+            raise ValueError("lse must be a contiguous float32 tensor of shape [B, Hq, L]")
+        p.lse = lse.data_ptr()
     if status is not None:
         p.status = status.data_ptr()
     rc = lib().krea_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),

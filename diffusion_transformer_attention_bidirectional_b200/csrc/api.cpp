@@ -592,6 +592,8 @@ int krea_attn_fwd(const void* q, const void* k, const void* v, const void* gate,
   ap.tma_out = tma_out ? 1 : 0;
   ap.wait_limit = p->debug_wait_limit > 0 ? p->debug_wait_limit : (long long)2000000000LL;
   ap.debug_flags = p->debug_flags;
+  if (p->lse && (reinterpret_cast<uintptr_t>(p->lse) & 3)) return KREA_ERR_INVALID_ARG;
+  ap.lse = p->lse;
   return launch_attention(ap, maps, bf16, stream);
 }
 

@@ -631,6 +631,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok) ok = wait_warp(ctl, bar(BAR_O + wg), 0);
       if (ok && staged && p.has_gate) ok = wait_warp(ctl, bar(BAR_GATE), 0);
+      if (ok && p.lse && q_valid)  // the softmax normaliser, natural log: (m + log2 l) ln 2
+        p.lse[((long long)b * p.Hq + h) * p.L + phys_q] = (m + log2f(l)) * 0.69314718055994531f;
       if (ok && staged) {
         // Staged epilogue: the gate row comes from the Q area (TMA-loaded, 64 values per
         // 128-byte swizzled row), out = O / l * sigmoid(gate) goes to the free K/V slots

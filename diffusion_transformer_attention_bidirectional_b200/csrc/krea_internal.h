@@ -91,6 +91,7 @@ struct AttnDevParams {
   int tma_out;         // out (and gate, when given) have TMA maps: staged epilogue allowed
   long long wait_limit;
   int debug_flags;
+  float* lse;          // [B, Hq, L] or null
 };
 
 struct QuantDevParams {

@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define KREA_ATTN_ABI_VERSION 1
+#define KREA_ATTN_ABI_VERSION 2
 #define KREA_ATTN_TILE 128
 
 typedef enum {
@@ -119,6 +119,9 @@ typedef struct {
   int64_t debug_wait_limit; /* SM clock cycles a kernel waits on one barrier before giving up; 0 -> 2e9 */
   int32_t debug_flags;   /* bit 0: one softmax warp waits on a barrier nothing arrives at (tests the bounded wait);
                             bit 1: every exponential through the FMA-pipe polynomial (tests its accuracy) */
+  float* lse;            /* optional device fp32 [B, Hq, L], 4-byte aligned: for every valid query row of the
+                            slice, ln sum_j exp(softmax_scale * s_ij) over its admitted keys (the softmax
+                            normaliser a backward pass needs); rows outside the slice are not written */
 } krea_attn_params_t;
 
 /* Fill `p` with the defaults for a contiguous [B, L, H, d] layout. */

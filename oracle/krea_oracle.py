@@ -340,7 +340,8 @@ def attention(case, q, k, v, gate=None, rows: Optional[Sequence[int]] = None,
     keys A(t) only. Scores s are FP16-tile scores q . k~ (k~ = centred keys
     under TileMix smooth_k) or INT8-tile scores s_q s_k (Q8 . K8), tile by tile
     as the map says. `rows` are physical query tokens (default: all).
-    Returns {"out": [B, R, Hq, d]} (+ "probs" [B, Hq, R, L] if asked).
+    Returns {"out": [B, R, Hq, d], "lse": [B, Hq, R]} (+ "probs" [B, Hq, R, L] if
+    asked); lse = log sum_{j in A(t)} exp(scale * s(t, j)), the softmax normaliser.
     """
     c = case
     qd, kd, vd, gd = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(gate)
@@ -380,6 +381,7 @@ def attention(case, q, k, v, gate=None, rows: Optional[Sequence[int]] = None,
 
     out = np.zeros((B, rows.shape[0], Hq, d))
     probs = np.zeros((B, Hq, rows.shape[0], L)) if return_probs else None
+    lse = np.zeros((B, Hq, rows.shape[0]))
     for b in batches:
         for h in heads:
             g = h // rep                                   # repeat_interleave order
@@ -393,14 +395,16 @@ def attention(case, q, k, v, gate=None, rows: Optional[Sequence[int]] = None,
             m = s.max(axis=1, keepdims=True)
             assert np.all(np.isfinite(m)), "a query row admits no key"
             p = np.exp(s - m)
-            p /= p.sum(axis=1, keepdims=True)
+            z = p.sum(axis=1, keepdims=True)
+            lse[b, h] = (m + np.log(z))[:, 0]
+            p /= z
             o = p @ vd[b, :, g, :]
             if gd is not None:
                 o = o * sigmoid(gd[b, rows, h, :])
             out[b, :, h, :] = o
             if return_probs:
                 probs[b, h] = p
-    res = {"out": out}
+    res = {"out": out, "lse": lse}
     if return_probs:
         res["probs"] = probs
     return res

@@ -303,3 +303,68 @@ def test_head_shards_equal_full_call():
                     window=7, out=os_)
     torch.cuda.synchronize()
     assert torch.equal(out, full)
+
+
+# ---------------------------------------------------------------------------- closed forms on the GPU path
+
+def test_single_admitted_key_returns_its_value():
+    # scanline, no text, one token per image row, window 1, token rule: every query
+    # admits exactly itself, so out = sigmoid(gate) * v (and v without a gate)
+    c = S.Case("one_key", 1, 4, 2, 128, 0, 300, 1, dtype="bf16", mode="scanline", seed=91, window=1,
+               tile_aligned=False)
+    q, k, v, _ = S.make_inputs(c)
+    out = gpu_run(c, q, k, v, None).cpu().numpy()
+    want = np.repeat(v.float().numpy(), 2, axis=2)  # q head h reads kv head h // 2
+    assert np.max(np.abs(out - want)) <= 1e-6 * max(1.0, float(np.max(np.abs(want))))
+    g = torch.from_numpy(np.random.default_rng(5).standard_normal(q.shape).astype(np.float32)).to(torch.bfloat16)
+    out_g = gpu_run(c, q, k, v, g).cpu().numpy()
+    sig = 1.0 / (1.0 + np.exp(-g.double().numpy()))
+    assert np.max(np.abs(out_g - sig * want)) <= 1e-5
+
+
+@pytest.mark.parametrize("mode,ta", [("dense", True), ("scanline", False), ("scanline", True)])
+def test_zero_queries_give_the_mean_of_admitted_values(mode, ta):
+    # q = 0: every admitted score is 0, every weight 1/|A(q)|; the admitted sets are
+    # written out here from the rule (text global, image rows within window // 2)
+    T, H, W, win = 130, 12, 20, 5
+    c = S.Case("qzero", 1, 2, 1, 128, T, H, W, dtype="bf16", mode=mode, seed=93, window=win, tile_aligned=ta)
+    _, k, v, _ = S.make_inputs(c)
+    q = torch.zeros(1, c.seq_len, 2, 128, dtype=torch.bfloat16)
+    out = gpu_run(c, q, k, v, None).cpu().numpy()[0, :, 0]
+    vv = v.double().numpy()[0, :, 0]
+    L = c.seq_len
+    for t in [0, 1, T - 1, T, T + 7, T + W * 5 + 3, L - 1]:
+        if mode == "dense" or t < T:
+            idx = np.arange(L)
+        else:
+            r = (t - T) // W
+            if ta:  # tile-aligned: every valid key of every active 128-tile pair
+                idx = None
+            else:
+                rows = range(max(0, r - win // 2), min(H, r + win // 2 + 1))
+                idx = np.r_[np.arange(T), [T + rr * W + cc for rr in rows for cc in range(W)]].astype(int)
+        if idx is None:
+            continue  # covered by the oracle comparisons; the rule above is per token
+        assert np.max(np.abs(out[t] - vv[idx].mean(axis=0))) <= 2e-6, t
+
+
+@pytest.mark.parametrize("mode", ["dense", "scanline", "tilemix"])
+def test_lse_matches_oracle(mode):
+    # the softmax normaliser ln sum_j exp(scale s_ij) per valid query row, written
+    # when asked for (the quantity a backward pass recomputes P from)
+    extra = dict(window=5, tile_aligned=False) if mode == "scanline" else {}
+    if mode == "tilemix":
+        extra = dict(pattern="band", percentage=0.5, band_blocks=1, smooth_k=True, qk_dist="normal_koffset")
+    c = S.Case("lse", 1, 4, 2, 128, 150, 14, 22, dtype="f16", mode=mode, seed=97, gate=True, **extra)
+    q, k, v, g = S.make_inputs(c)
+    lse = torch.full((1, 4, c.seq_len), float("nan"), dtype=torch.float32, device="cuda")
+    out = gpu_run(c, q, k, v, g, lse=lse)
+    ref = ko.attention(c, q, k, v, g)
+    tol = 1e-3 if mode == "tilemix" else 1e-4
+    assert np.max(np.abs(lse.cpu().numpy() - ref["lse"])) <= tol
+    # a slice writes only its own rows
+    lse2 = torch.full_like(lse, float("nan"))
+    gpu_run(c, q, k, v, g, lse=lse2, q_start=128, q_len=200)
+    got = lse2.cpu().numpy()
+    assert np.all(np.isnan(got[..., :128])) and np.all(np.isnan(got[..., 328:]))
+    assert np.max(np.abs(got[..., 128:328] - ref["lse"][..., 128:328])) <= tol
