@@ -410,6 +410,43 @@ def attention(case, q, k, v, gate=None, rows: Optional[Sequence[int]] = None,
     return res
 
 
+def attention_backward(case, q, k, v, gate, dout) -> Dict[str, np.ndarray]:
+    """Gradients of out = sigmoid(gate) * softmax(scale * q k^T over A) v with respect
+    to q, k, v and gate, given dout [B, L, Hq, d]; FP16-tile scores only (dense and
+    scanline: the INT8 codes of TileMix have no gradient).
+
+    With P the softmax weights over the admitted keys and O = P v (before the gate):
+      dO = dout * sigmoid(g);  dgate = dout * O * sigmoid(g) (1 - sigmoid(g))
+      dV_j = sum_i P_ij dO_i;   dP_ij = dO_i . v_j;   D_i = sum_j P_ij dP_ij = dO_i . O_i
+      dS_ij = P_ij (dP_ij - D_i);  dQ_i = scale sum_j dS_ij k_j;  dK_j = scale sum_i dS_ij q_i
+    summed over the rep query heads that share a kv head for dK and dV.
+    """
+    c = case
+    assert c.mode != "tilemix" or c.pattern == "zero", "INT8 tiles have no gradient"
+    qd, kd, vd, gd, dod = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(gate), _as_f64(dout)
+    B, L, Hq, d = qd.shape
+    rep = Hq // kd.shape[2]
+    scale = c.softmax_scale if c.softmax_scale else 1.0 / math.sqrt(d)
+    fwd = attention(c, q, k, v, None, return_probs=True)
+    O = fwd["out"]                                   # before the gate
+    P = fwd["probs"]                                 # [B, Hq, L, L], zero off the admitted set
+    dq, dk, dv = np.zeros_like(qd), np.zeros_like(kd), np.zeros_like(vd)
+    sg = sigmoid(gd) if gd is not None else None
+    dO = dod * sg if gd is not None else dod
+    dgate = dod * O * sg * (1.0 - sg) if gd is not None else None
+    for b in range(B):
+        for h in range(Hq):
+            g = h // rep
+            p = P[b, h]
+            dv[b, :, g, :] += p.T @ dO[b, :, h, :]
+            dp = dO[b, :, h, :] @ vd[b, :, g, :].T
+            Dr = np.sum(dO[b, :, h, :] * O[b, :, h, :], axis=1, keepdims=True)
+            ds = p * (dp - Dr)
+            dq[b, :, h, :] = scale * ds @ kd[b, :, g, :]
+            dk[b, :, g, :] += scale * ds.T @ qd[b, :, h, :]
+    return {"dq": dq, "dk": dk, "dv": dv, "dgate": dgate}
+
+
 # ----------------------------------------------------------------------------
 # QK prologue: RMSNorm, then the 3-axis rotary embedding
 # ----------------------------------------------------------------------------

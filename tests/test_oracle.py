@@ -428,3 +428,51 @@ def test_qk_prologue_is_norm_then_rope():
     # rotation keeps each pair's length, so the RMS of y is that of the normalised x
     assert np.allclose(np.mean(y * y, -1), np.mean(ko.rms_norm(x, g) ** 2, -1), atol=1e-12)
     assert np.allclose(y[:, 0], ko.rms_norm(x, g)[:, 0], atol=0)  # token 0 sits at (0, 0, 0)
+
+
+# ---------------------------------------------------------------------------- backward pins
+
+def _loss(c, q, k, v, g, w):
+    return float(np.sum(ko.attention(c, q, k, v, g)["out"] * w))
+
+
+@pytest.mark.parametrize("mode,extra", [("dense", {}), ("scanline", dict(window=3, tile_aligned=False)),
+                                        ("scanline", dict(window=3, tile_aligned=True))])
+def test_backward_matches_central_differences(mode, extra):
+    # d/dx of sum(out * w) by central differences on a tiny case, every input entry
+    # of a few sampled coordinates: pins every term of the backward formulas
+    c = Case("bw", 1, 2, 1, 8, 3, 3, 4, mode=mode, seed=12, softmax_scale=0.7, **extra)
+    rng = np.random.default_rng(4)
+    L = c.seq_len
+    q, k, v = (rng.standard_normal((1, L, h, 8)) for h in (2, 1, 1))
+    g = rng.standard_normal((1, L, 2, 8))
+    w = rng.standard_normal((1, L, 2, 8))
+    grads = ko.attention_backward(c, q, k, v, g, w)
+    eps = 1e-6
+    for name, x in (("dq", q), ("dk", k), ("dv", v), ("dgate", g)):
+        idx = [tuple(rng.integers(0, n) for n in x.shape) for _ in range(12)]
+        for ix in idx:
+            xp, xm = x.copy(), x.copy()
+            xp[ix] += eps
+            xm[ix] -= eps
+            args = {"dq": (xp, k, v, g), "dk": (q, xp, v, g), "dv": (q, k, xp, g), "dgate": (q, k, v, xp)}[name]
+            argm = {"dq": (xm, k, v, g), "dk": (q, xm, v, g), "dv": (q, k, xm, g), "dgate": (q, k, v, xm)}[name]
+            num = (_loss(c, *args, w) - _loss(c, *argm, w)) / (2 * eps)
+            assert abs(num - grads[name][ix]) <= 1e-6 * max(1.0, abs(num)), (name, ix, num, grads[name][ix])
+
+
+def test_backward_closed_forms():
+    # dV_j = sum_i P_ij dO_i: with q = 0 (dense) every weight is 1 / L, so every row of
+    # dV is the sum of dO over all queries and both heads of the group, divided by L
+    c = Case("bw2", 1, 2, 1, 8, 0, 4, 5, mode="dense", seed=13)
+    rng = np.random.default_rng(6)
+    L = c.seq_len
+    q = np.zeros((1, L, 2, 8))
+    k, v = rng.standard_normal((1, L, 1, 8)), rng.standard_normal((1, L, 1, 8))
+    w = rng.standard_normal((1, L, 2, 8))
+    gr = ko.attention_backward(c, q, k, v, None, w)
+    want_dv = (w[0, :, 0, :].sum(0) + w[0, :, 1, :].sum(0)) / L
+    assert np.allclose(gr["dv"][0, :, 0, :], want_dv[None, :], atol=1e-12)
+    # a row's weights do not change when every key moves by the same vector (each
+    # score of the row shifts by one constant): sum_j dS_ij = 0, so sum_j dK_j = 0
+    assert np.allclose(gr["dk"].sum(axis=1), 0.0, atol=1e-12)
