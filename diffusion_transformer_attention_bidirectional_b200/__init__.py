@@ -231,6 +231,41 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[
     return out
 
 
+def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[torch.Tensor],
+                       out: torch.Tensor, dout: torch.Tensor, lse: torch.Tensor, *, text_len: int, grid_h: int,
+                       grid_w: int, mode: str = "dense", stream: Optional[torch.cuda.Stream] = None,
+                       status: Optional[torch.Tensor] = None, **opts):
+    """(dq, dk, dv, dgate) of krea_attn_fwd's output (fp32 tensors; dgate None without
+    a gate). out, dout: the forward's output and its gradient, contiguous, same dtype;
+    lse: the forward's [B, Hq, L] log-sum-exp (attention(..., lse=...))."""
+    _check_inputs(q, k, v, gate, out, dout, lse, status)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    in_dt = _TORCH_DT[q.dtype]
+    p = make_params(B, Hq, Hkv, d, text_len, grid_h, grid_w, in_dtype=in_dt, out_dtype=_TORCH_DT[out.dtype],
+                    **opts)
+    for arr, t in ((p.q_stride, q), (p.k_stride, k), (p.v_stride, v)):
+        arr[0], arr[1], arr[2] = t.stride()[:3]
+    if gate is not None:
+        p.gate_stride[0], p.gate_stride[1], p.gate_stride[2] = gate.stride()[:3]
+    if status is not None:
+        p.status = status.data_ptr()
+    out, dout = out.contiguous(), dout.contiguous()
+    dq = torch.empty(B, L, Hq, d, dtype=torch.float32, device=q.device)
+    dk = torch.empty(B, L, Hkv, d, dtype=torch.float32, device=q.device)
+    dv = torch.empty(B, L, Hkv, d, dtype=torch.float32, device=q.device)
+    dgate = torch.empty(B, L, Hq, d, dtype=torch.float32, device=q.device) if gate is not None else None
+    scratch = torch.empty(int(lib().krea_attn_bwd_scratch_bytes(text_len, grid_h, grid_w, ctypes.byref(p))),
+                          dtype=torch.uint8, device=q.device)
+    check(lib().krea_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                              gate.data_ptr() if gate is not None else None, out.data_ptr(), dout.data_ptr(),
+                              lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                              dgate.data_ptr() if dgate is not None else None, scratch.data_ptr(),
+                              text_len, grid_h, grid_w, _lib.MODE[mode], ctypes.byref(p),
+                              _stream_ptr(stream, q.device)), "krea_attn_bwd")
+    return dq, dk, dv, dgate
+
+
 def quantize(q: torch.Tensor, k: torch.Tensor, *, text_len: int, grid_h: int, grid_w: int,
              smooth_k: bool = True, workspace: Optional[torch.Tensor] = None,
              stream: Optional[torch.cuda.Stream] = None) -> dict:

@@ -597,6 +597,96 @@ int krea_attn_fwd(const void* q, const void* k, const void* v, const void* gate,
   return launch_attention(ap, maps, bf16, stream);
 }
 
+size_t krea_attn_bwd_scratch_bytes(int text_len, int grid_h, int grid_w, const krea_attn_params_t* p) {
+  if (check_common(p) != KREA_OK) return 0;
+  const size_t L = (size_t)text_len + (size_t)grid_h * grid_w;
+  const size_t dO = align256(L * p->batch * p->num_q_heads * p->head_dim * elem_bytes(p->in_dtype));
+  return dO + align256(L * p->batch * p->num_q_heads * sizeof(float));
+}
+
+int krea_attn_bwd(const void* q, const void* k, const void* v, const void* gate, const void* out, const void* dout,
+                  const float* lse, float* dq, float* dk, float* dv, float* dgate, void* scratch, int text_len,
+                  int grid_h, int grid_w, int mode, const krea_attn_params_t* p, void* stream) {
+  int rc = check_common(p);
+  if (rc != KREA_OK) return rc;
+  if (mode == KREA_MODE_TILEMIX) return KREA_ERR_UNSUPPORTED;
+  Geometry g;
+  rc = make_geometry(text_len, grid_h, grid_w, mode, p, &g);
+  if (rc != KREA_OK) return rc;
+  if (p->q_start != 0 || (p->q_len != 0 && p->q_len != g.L)) return KREA_ERR_UNSUPPORTED;
+  const int es = elem_bytes(p->in_dtype);
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !scratch) return KREA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, out, dout, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return KREA_ERR_INVALID_ARG;
+  if ((gate && !aligned16(gate)) || (dgate && !aligned16(dgate)) || (reinterpret_cast<uintptr_t>(scratch) & 255))
+    return KREA_ERR_INVALID_ARG;
+  if (!stride_ok(p->q_stride, es) || !stride_ok(p->k_stride, es) || !stride_ok(p->v_stride, es) ||
+      (gate && !stride_ok(p->gate_stride, es)))
+    return KREA_ERR_INVALID_ARG;
+  rc = check_device();
+  if (rc != KREA_OK) return rc;
+  MapEntry map;
+  rc = get_device_map(g, &map);
+  if (rc != KREA_OK) return rc;
+  const int B = p->batch, Hq = p->num_q_heads, Hkv = p->num_kv_heads, d = p->head_dim;
+  char* sc = static_cast<char*>(scratch);
+  void* dO = sc;
+  float* D = reinterpret_cast<float*>(sc + align256((size_t)g.L * B * Hq * d * es));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(dq, 0, (size_t)B * g.L * Hq * d * sizeof(float), s) != cudaSuccess) return KREA_ERR_CUDA;
+  BwdPrepParams pp;
+  pp.out = out;
+  pp.dout = dout;
+  pp.gate = gate;
+  for (int i = 0; i < 3; ++i) pp.g_stride[i] = p->gate_stride[i];
+  pp.dO = dO;
+  pp.D = D;
+  pp.dgate = gate ? dgate : nullptr;
+  pp.B = B;
+  pp.L = g.L;
+  pp.H = Hq;
+  pp.d = d;
+  const bool bf16 = p->in_dtype == KREA_BF16;
+  rc = launch_bwd_prep(pp, bf16, p->out_dtype == KREA_F32, stream);
+  if (rc != KREA_OK) return rc;
+  const CUtensorMapDataType tdt = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  BwdMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const int64_t dO_stride[3] = {(int64_t)g.L * Hq * d, (int64_t)Hq * d, (int64_t)d};
+  rc = make_tmap(&maps.q, q, tdt, es, d, Hq, g.L, B, p->q_stride, 64);
+  if (rc == KREA_OK) rc = make_tmap(&maps.k, k, tdt, es, d, Hkv, g.L, B, p->k_stride, 64);
+  if (rc == KREA_OK) rc = make_tmap(&maps.v, v, tdt, es, d, Hkv, g.L, B, p->v_stride, 64);
+  if (rc == KREA_OK) rc = make_tmap(&maps.dout, dO, tdt, es, d, Hq, g.L, B, dO_stride, 64);
+  if (rc != KREA_OK) return rc;
+  BwdDevParams bp;
+  bp.row_ptr = map.d_row_ptr;
+  bp.entries = map.d_entries;
+  bp.lse = lse;
+  bp.D = D;
+  bp.dq = dq;
+  bp.dk = dk;
+  bp.dv = dv;
+  bp.status = p->status;
+  bp.B = B;
+  bp.Hq = Hq;
+  bp.Hkv = Hkv;
+  bp.d = d;
+  bp.rep = Hq / Hkv;
+  bp.T = g.T;
+  bp.N = g.N;
+  bp.Pt = g.Pt;
+  bp.L = g.L;
+  bp.W = g.W;
+  bp.H = g.H;
+  bp.window_half = g.window / 2;
+  bp.tile_aligned = (mode != KREA_MODE_SCANLINE) || g.tile_aligned;
+  bp.n_tiles = g.n_tiles;
+  bp.scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt((float)d);
+  bp.scale_log2 = bp.scale * 1.4426950408889634f;
+  bp.wait_limit = p->debug_wait_limit > 0 ? p->debug_wait_limit : (long long)2000000000LL;
+  return launch_backward(bp, maps, bf16, stream);
+}
+
 void krea_attn_clear_cache(void) {
   std::lock_guard<std::mutex> lock(g_cache_mu);
   for (auto& e : g_cache) free_entry(e);

@@ -65,6 +65,35 @@ struct PrologueDevParams {
 int launch_rope_table(const int32_t* pos, int tokens, const int axes[3], double theta, float* table, void* stream);
 int launch_prologue(const PrologueDevParams& p, bool bf16, void* stream);
 
+// Backward (bwd.cu).
+struct alignas(64) BwdMaps { CUtensorMap q, k, v, dout; };  // dout: the dO scratch tensor
+struct BwdDevParams {
+  const int32_t* row_ptr;
+  const int32_t* entries;
+  const float* lse;     // [B, Hq, L] natural log
+  const float* D;       // [B, Hq, L]
+  float* dq;            // [B, L, Hq, d] fp32, accumulated (zeroed by the host)
+  float* dk;            // [B, L, Hkv, d] fp32
+  float* dv;            // [B, L, Hkv, d] fp32
+  int32_t* status;
+  int B, Hq, Hkv, d, rep;
+  int T, N, Pt, L, W, H, window_half, tile_aligned, n_tiles;
+  float scale, scale_log2;
+  long long wait_limit;
+};
+struct BwdPrepParams {
+  const void* out;      // [B, L, Hq, d], fp32 or the input dtype, contiguous
+  const void* dout;     // same type and layout as out
+  const void* gate;     // input dtype or null
+  long long g_stride[3];
+  void* dO;             // [B, L, Hq, d] input dtype, contiguous
+  float* D;             // [B, Hq, L]
+  float* dgate;         // [B, L, Hq, d] fp32 or null
+  int B, L, H, d;
+};
+int launch_bwd_prep(const BwdPrepParams& p, bool bf16, bool out32, void* stream);
+int launch_backward(const BwdDevParams& p, const BwdMaps& m, bool bf16, void* stream);
+
 // Resolves and validates the geometry of a call.
 int make_geometry(int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* p,
                   Geometry* g);

@@ -240,6 +240,25 @@ KREA_API int krea_attn_fwd_noalloc(const void* q, const void* k, const void* v, 
                                    int text_len, int grid_h, int grid_w, int mode,
                                    const krea_attn_params_t* params, void* stream);
 
+/* Backward of krea_attn_fwd for dense and scanline calls (TileMix INT8 codes
+ * have no gradient): with P the softmax weights over the admitted keys (from the
+ * forward's lse), O = P v and out = sigmoid(gate) O,
+ *   dv = P^T dO, dq = scale dS k, dk = scale dS^T q, dgate = dout out (1 - sigmoid(gate)),
+ *   dO = dout sigmoid(gate), dS = P (dO v^T - rowsum(dout out)),
+ * dk and dv summed over the query heads of each kv head.
+ * Inputs: q, k, v, gate as given to the forward (params strides and dtype), out
+ * and dout contiguous [B, L, Hq, d] of params->out_dtype, lse [B, Hq, L] fp32 from
+ * the forward (params->lse). Outputs, all fp32 and contiguous: dq [B, L, Hq, d]
+ * (zeroed, then accumulated), dk and dv [B, L, Hkv, d], dgate [B, L, Hq, d] (may
+ * be NULL; ignored without a gate). scratch: krea_attn_bwd_scratch_bytes() bytes
+ * of device memory, 256-byte aligned. The whole sequence only (q_start 0, q_len 0
+ * or L); head_dim 64 or 128. */
+KREA_API size_t krea_attn_bwd_scratch_bytes(int text_len, int grid_h, int grid_w, const krea_attn_params_t* params);
+KREA_API int krea_attn_bwd(const void* q, const void* k, const void* v, const void* gate, const void* out,
+                           const void* dout, const float* lse, float* dq, float* dk, float* dv, float* dgate,
+                           void* scratch, int text_len, int grid_h, int grid_w, int mode,
+                           const krea_attn_params_t* params, void* stream);
+
 /* Release every cached tile map on every device. */
 KREA_API void krea_attn_clear_cache(void);
 
