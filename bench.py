@@ -240,6 +240,35 @@ def time_prologue(K, device, stream, flush, P, reps: int = 8):
             "bound": "hbm", "peak_source": f"{P['source']} copy bandwidth", "l2": "flushed before each pass"}
 
 
+def time_backward(K, device, stream, flush, P, reps: int = 6):
+    """The backward (prep + dq/dk/dv kernel) on the dense 1 MP shape: 48/12 heads,
+    d 128, bf16, gate. Algorithmic FLOPs: five products of 2 d per admitted pair
+    (S, dP, dV, dK, dQ), i.e. 10 d per pair per query head."""
+    from synth import inputs as S
+
+    c = S.dense_1mp()
+    q, k, v, g = (t.to(device) for t in S.make_inputs(c))
+    lse = torch.empty(c.batch, c.q_heads, c.seq_len, dtype=torch.float32, device=device)
+    out = K.attention(q, k, v, g, text_len=c.text_len, grid_h=c.grid_h, grid_w=c.grid_w, lse=lse)
+    dout = torch.randn(out.shape, dtype=torch.float32, device=device, generator=torch.Generator(device).manual_seed(7))
+    times = []
+    for it in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        K.attention_backward(q, k, v, g, out, dout, lse, text_len=c.text_len, grid_h=c.grid_h, grid_w=c.grid_w)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        if it >= 2:
+            times.append(a.elapsed_time(b))
+    ms = sorted(times)[len(times) // 2]
+    flops = 10.0 * c.batch * c.q_heads * c.head_dim * c.seq_len * c.seq_len
+    return {"workload": "dense 1 MP backward: B=1, 48/12 heads, d=128, 512 text + 64x64, bf16, gate",
+            "ms": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+            "frac_of_peak": round(flops / (ms * 1e-3) / 1e12 / P["bf16"], 4),
+            "note": "includes dq zeroing, the prep pass and the scratch allocation of the Python wrapper"}
+
+
 def run_ours(args, rank, world, device):
     import diffusion_transformer_attention_bidirectional_b200 as K
     from synth import inputs as S
@@ -419,6 +448,7 @@ def run_ours(args, rank, world, device):
         raise RuntimeError(f"device status {int(status.item())} during the comparisons")
 
     prologue = None if args.no_comparisons else time_prologue(K, device, stream, flush, P)
+    backward = None if args.no_comparisons else time_backward(K, device, stream, flush, P)
 
     # roofline of the dominant kernel: the attention kernel on the dense variant
     # (its launches are attention kernels only), algorithmic FLOPs / event time
@@ -466,6 +496,8 @@ def run_ours(args, rank, world, device):
     }
     if prologue is not None:
         res["prologue"] = prologue
+    if backward is not None:
+        res["backward"] = backward
     dense_tf = next((v["tflops"] for n, v in variants.items() if "cfg_pair" in n), None)
     for n, v in variants.items():
         if dense_tf and n.startswith("scanline"):

@@ -54,3 +54,28 @@ def test_backward_scanline(ta):
     c = S.Case("bwd_scan", 2, 4, 1, 128, 100, 12, 20, dtype="bf16", mode="scanline", seed=111, window=3,
                tile_aligned=ta)
     run_case(c, True)
+
+
+def test_backward_full_size_one_group():
+    # the dense 1 MP workload (48/12 heads) through the backward; kv-head groups are
+    # independent, so group 5 must equal the oracle run on that group alone
+    c = S.dense_1mp()
+    q, k, v, g = S.make_inputs(c)
+    dev = torch.device("cuda:0")
+    lse = torch.empty(1, 48, c.seq_len, dtype=torch.float32, device=dev)
+    qd, kd, vd, gd = q.to(dev), k.to(dev), v.to(dev), g.to(dev)
+    out = K.attention(qd, kd, vd, gd, text_len=c.text_len, grid_h=c.grid_h, grid_w=c.grid_w, lse=lse)
+    w = torch.from_numpy(np.random.default_rng(3).standard_normal(out.shape).astype(np.float32))
+    dq, dk, dv, dgate = K.attention_backward(qd, kd, vd, gd, out, w.to(dev), lse, text_len=c.text_len,
+                                             grid_h=c.grid_h, grid_w=c.grid_w)
+    torch.cuda.synchronize()
+    grp = 5
+    hs = slice(4 * grp, 4 * grp + 4)
+    sub = S.Case("grp", 1, 4, 1, 128, c.text_len, c.grid_h, c.grid_w, dtype="bf16", mode="dense", seed=0)
+    ref = ko.attention_backward(sub, q[:, :, hs], k[:, :, grp:grp + 1], v[:, :, grp:grp + 1], g[:, :, hs],
+                                w[:, :, hs])
+    for name, x in (("dq", dq[:, :, hs]), ("dk", dk[:, :, grp:grp + 1]), ("dv", dv[:, :, grp:grp + 1]),
+                    ("dgate", dgate[:, :, hs])):
+        r = ref[name]
+        err = float(np.max(np.abs(x.cpu().numpy() - r)))
+        assert err <= 8 * EPS["bf16"] * float(np.max(np.abs(r))), (name, err)
