@@ -11,7 +11,8 @@
 // bwd_kernel: one CTA per (batch, kv head, key tile j), 192 threads:
 //   warps 0-3  thread = query row of the current query tile (P and dS), then key
 //              row of tile j (writes dK, dV at the end)
-//   warp  4    TMA producer: K_j and V_j once, then Q_i, dO_i per step
+//   warp  4    TMA producer: K_j and V_j once, then Q_i, dO_i per step (as soon
+//              as dV and dK of the previous step have read them)
 //   warp  5    TMEM allocator and the thread issuing every tcgen05.mma
 // A step is one (query head, query tile i) of the key tile's map row (the
 // scanline rule is symmetric, so row j lists the query tiles that see tile j):
@@ -41,7 +42,7 @@ constexpr int kBThreads = 192;
 constexpr uint32_t kBBox = 16384;        // 128 rows x 128 bytes
 constexpr uint32_t BS_K = 0, BS_V = 32768, BS_Q = 65536, BS_DO = 98304, BS_P = 131072, BS_DS = 163840;
 constexpr uint32_t BS_BAR = 196608;
-enum { BB_KV = 0, BB_QF, BB_SDP, BB_PDS, BB_GRAD, BB_SFREE, BB_DRAIN, BB_N };
+enum { BB_KV = 0, BB_QF, BB_SDP, BB_PDS, BB_GRAD, BB_SFREE, BB_DRAIN, BB_QFREE, BB_N };
 constexpr uint32_t BS_TMEM = BS_BAR + 8 * BB_N;
 constexpr uint32_t BS_ABORT = BS_TMEM + 4;
 constexpr uint32_t B_SMEM_ALLOC = BS_BAR + 128 + 1024;  // + slack to align the base to 1024
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     ptx::mbar_init(bar(BB_GRAD), 1);
     ptx::mbar_init(bar(BB_SFREE), 4);
     ptx::mbar_init(bar(BB_DRAIN), 1);
+    ptx::mbar_init(bar(BB_QFREE), 1);
     *abort_flag = 0;
     ptx::fence_barrier_init();
     ptx::fence_proxy_async_smem();
@@ -170,7 +172,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
       }
       int s = 0;
       for (; s < nsteps; ++s) {
-        if (s > 0 && !b_wait1(ctl, bar(BB_GRAD), (s - 1) & 1)) break;  // step s-1 has read Q, dO
+        if (s > 0 && !b_wait1(ctl, bar(BB_QFREE), (s - 1) & 1)) break;  // dV, dK of s-1 read Q, dO
         const int h = g * p.rep + s / n;
         const int qrow0 = b_row0(p.entries[e0 + s % n] >> 2, p);
         ptx::mbar_arrive_expect_tx(bar(BB_QF), 2 * nbox * kBBox);
@@ -218,6 +220,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
           ptx::mma_f16_ss_lo(tmem + 256u, mP + 128u * k, mDO + 128u * k, ID_MM, acc);   // dV += P^T dO
           ptx::mma_f16_ss_lo(tmem + 384u, mDS + 128u * k, mQ + 128u * k, ID_MM, acc);   // dK += dS^T Q
         }
+        ptx::tc_commit(bar(BB_QFREE));  // Q and dO may be replaced while dQ is formed
         for (int k = 0; k < 8; ++k) {  // dQ part = dS K_j, K = 128 keys
           const uint32_t off = (uint32_t)(k >> 2) * kb4 + (uint32_t)(k & 3) * 2u;
           ptx::mma_f16_ss_lo(tmem, dS_k + off, mK + 128u * k, ID_KM, k > 0);
