@@ -579,6 +579,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prologue-only", action="store_true",
                     help="time only the QK prologue at the 4 MP shape (profiling)")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the backward at the dense 1 MP shape (profiling)")
     ap.add_argument("--no-comparisons", action="store_true",
                     help="skip the band-vs-zero timing after the timed steps (launch-list captures)")
     ap.add_argument("--case", default=None,
@@ -605,12 +607,13 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
-    if args.prologue_only:
+    if args.prologue_only or args.backward_only:
         import diffusion_transformer_attention_bidirectional_b200 as K
 
         torch.cuda.set_device(device)
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
-        print(json.dumps(time_prologue(K, device, torch.cuda.current_stream(device), flush, peaks())), flush=True)
+        fn = time_prologue if args.prologue_only else time_backward
+        print(json.dumps(fn(K, device, torch.cuda.current_stream(device), flush, peaks())), flush=True)
         return
     try:
         res = run_ours(args, rank, world, device)
