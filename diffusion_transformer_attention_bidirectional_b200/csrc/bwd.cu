@@ -295,22 +295,29 @@ __global__ void __launch_bounds__(kBThreads, 1)
       if (!ok) break;
       ptx::tc_fence_after();
       float* dqrow = p.dq + (((long long)b * p.L + (q_valid ? phys_q : 0)) * p.Hq + h) * d;
-      for (int c32 = 0; c32 < d / 32; ++c32) {
-        uint32_t o[32];
-        __syncwarp();
-        ptx::tmem_ld32(tS + 32u * c32, o);
-        ptx::tmem_wait_ld();
-        if (q_valid) {
-#pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4)
-            red_add_v4(dqrow + 32 * c32 + 4 * v4, __uint_as_float(o[4 * v4]) * p.scale,
-                       __uint_as_float(o[4 * v4 + 1]) * p.scale, __uint_as_float(o[4 * v4 + 2]) * p.scale,
-                       __uint_as_float(o[4 * v4 + 3]) * p.scale);
-        }
+      // the whole dQ row into registers first, then free the TMEM columns, then add
+      // into dq: an arrive orders this thread's earlier memory operations, so the
+      // reductions come after it and the MMA thread never waits on their round trip
+      uint32_t dqv[128];
+      __syncwarp();
+      ptx::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&dqv[0]));
+      ptx::tmem_ld32(tS + 32u, *reinterpret_cast<uint32_t(*)[32]>(&dqv[32]));
+      if (d == 128) {
+        ptx::tmem_ld32(tS + 64u, *reinterpret_cast<uint32_t(*)[32]>(&dqv[64]));
+        ptx::tmem_ld32(tS + 96u, *reinterpret_cast<uint32_t(*)[32]>(&dqv[96]));
       }
+      ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(BB_SFREE));
+      if (q_valid) {
+#pragma unroll
+        for (int v4 = 0; v4 < 32; ++v4)
+          if (4 * v4 < d)
+            red_add_v4(dqrow + 4 * v4, __uint_as_float(dqv[4 * v4]) * p.scale,
+                       __uint_as_float(dqv[4 * v4 + 1]) * p.scale, __uint_as_float(dqv[4 * v4 + 2]) * p.scale,
+                       __uint_as_float(dqv[4 * v4 + 3]) * p.scale);
+      }
     }
     if (ok) {
       // dK and dV of key tile j, row = key row: the last GRAD commit covers every MMA
