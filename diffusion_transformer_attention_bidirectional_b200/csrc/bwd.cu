@@ -8,12 +8,15 @@
 // dK and dV summed over the query heads that share a kv head.
 //
 // bwd_prep_kernel: dO (input dtype), D and dgate, one pass over out / dout.
-// bwd_kernel: one CTA per (batch, kv head, key tile j), 192 threads:
-//   warps 0-3  thread = query row of the current query tile (P and dS), then key
-//              row of tile j (writes dK, dV at the end)
-//   warp  4    TMA producer: K_j and V_j once, then Q_i, dO_i per step (as soon
+// bwd_kernel: one CTA per (batch, kv head, key tile j), 320 threads:
+//   warps 0-7  warp w: TMEM lanes 32 (w % 4) .. (query rows of the current query
+//              tile, key rows of tile j at the end) and key / head-dim columns
+//              [64 (w / 4), + 64): P and dS need no row-wide reduction (the
+//              forward's lse and D are per-row constants), so the two warps of a
+//              row work independently
+//   warp  8    TMA producer: K_j and V_j once, then Q_i, dO_i per step (as soon
 //              as dV and dK of the previous step have read them)
-//   warp  5    TMEM allocator and the thread issuing every tcgen05.mma
+//   warp  9    TMEM allocator and the thread issuing every tcgen05.mma
 // A step is one (query head, query tile i) of the key tile's map row (the
 // scanline rule is symmetric, so row j lists the query tiles that see tile j):
 //   S = Q_i K_j^T, dP = dO_i V_j^T                 (TMEM columns 0..127, 128..255)
@@ -38,7 +41,7 @@
 namespace krea {
 namespace {
 
-constexpr int kBThreads = 192;
+constexpr int kBThreads = 320;
 constexpr uint32_t kBBox = 16384;        // 128 rows x 128 bytes
 constexpr uint32_t BS_K = 0, BS_V = 32768, BS_Q = 65536, BS_DO = 98304, BS_P = 131072, BS_DS = 163840;
 constexpr uint32_t BS_BAR = 196608;
@@ -141,16 +144,16 @@ __global__ void __launch_bounds__(kBThreads, 1)
     ptx::mbar_init(bar(BB_KV), 1);
     ptx::mbar_init(bar(BB_QF), 1);
     ptx::mbar_init(bar(BB_SDP), 1);
-    ptx::mbar_init(bar(BB_PDS), 4);
+    ptx::mbar_init(bar(BB_PDS), 8);
     ptx::mbar_init(bar(BB_GRAD), 1);
-    ptx::mbar_init(bar(BB_SFREE), 4);
+    ptx::mbar_init(bar(BB_SFREE), 8);
     ptx::mbar_init(bar(BB_DRAIN), 1);
     ptx::mbar_init(bar(BB_QFREE), 1);
     *abort_flag = 0;
     ptx::fence_barrier_init();
     ptx::fence_proxy_async_smem();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_ptr), 512);
     ptx::tmem_relinquish();
   }
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const int d = p.d;
   const int nbox = d / 64;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
       const int krow0 = b_row0(j, p);
@@ -185,7 +188,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
       b_drain(bar(BB_KV), 0);
       if (s > 0) b_drain(bar(BB_QF), (s - 1) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t ab = BF16 ? 1u : 0u;
@@ -232,10 +235,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
     }
   } else {
     // ------------------------------------------------------------- softmax warps
-    const int wq = warp, row = wq * 32 + lane;
+    const int wq = warp & 3, hf = warp >> 2, row = wq * 32 + lane;
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_base, tP = tS + 128u, tdV = tS + 256u, tdK = tS + 384u;
     const uint32_t rsw = (uint32_t)(row & 7), rofs = (uint32_t)row * 128u;
+    const int hd0 = hf * (d / 2);  // this warp's head-dim columns of dQ, dK, dV: [hd0, hd0 + d/2)
     bool ok = true;
     for (int s = 0; s < nsteps && ok; ++s) {
       const int hh = s / n, h = g * p.rep + hh;
@@ -255,24 +259,22 @@ __global__ void __launch_bounds__(kBThreads, 1)
       ok = b_wait_warp(ctl, bar(BB_SDP), s & 1);
       if (!ok) break;
       ptx::tc_fence_after();
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t sv[64], dp[64];
+      for (int ck = 0; ck < 2; ++ck) {  // keys 64 hf + 32 ck .. + 31 of S and dP -> P and dS
+        uint32_t sv[32], dp[32];
         __syncwarp();
-        ptx::tmem_ld32(tS + 64u * hf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        ptx::tmem_ld32(tS + 64u * hf + 32u, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        ptx::tmem_ld32(tP + 64u * hf, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        ptx::tmem_ld32(tP + 64u * hf + 32u, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        ptx::tmem_ld32(tS + 64u * hf + 32u * ck, sv);
+        ptx::tmem_ld32(tP + 64u * hf + 32u * ck, dp);
         ptx::tmem_wait_ld();
-        const int ks0 = j * kTile + 64 * hf;  // logical slot of this half's first key
+        const int ks0 = j * kTile + 64 * hf + 32 * ck;  // logical slot of the chunk's first key
 #pragma unroll
-        for (int piece = 0; piece < 8; ++piece) {  // 8 keys = 16 bytes of P and of dS
+        for (int pc = 0; pc < 4; ++pc) {  // 8 keys = 16 bytes of P and of dS
           uint32_t pw[4], dw[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             float pr[2], dr[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int c = piece * 8 + 2 * u + e;
+              const int c = pc * 8 + 2 * u + e;
               const int ks = ks0 + c;
               const bool adm = q_valid && (ks < p.T || (ks >= klo && ks < khi));
               const float pv = adm ? ptx::ex2(__uint_as_float(sv[c]) * p.scale_log2 - lse2) : 0.f;
@@ -282,7 +284,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
             pw[u] = b_pack<BF16>(pr[0], pr[1]);
             dw[u] = b_pack<BF16>(dr[0], dr[1]);
           }
-          const uint32_t at = (uint32_t)hf * kBBox + rofs + (((uint32_t)piece ^ rsw) << 4);
+          const uint32_t piece = (uint32_t)(4 * ck + pc);  // 16-byte piece of the 128-byte row
+          const uint32_t at = (uint32_t)hf * kBBox + rofs + ((piece ^ rsw) << 4);
           *reinterpret_cast<uint4*>(sb + BS_P + at) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
           *reinterpret_cast<uint4*>(sb + BS_DS + at) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
         }
@@ -294,35 +297,33 @@ __global__ void __launch_bounds__(kBThreads, 1)
       ok = b_wait_warp(ctl, bar(BB_GRAD), s & 1);
       if (!ok) break;
       ptx::tc_fence_after();
-      float* dqrow = p.dq + (((long long)b * p.L + (q_valid ? phys_q : 0)) * p.Hq + h) * d;
-      // the whole dQ row into registers first, then free the TMEM columns, then add
-      // into dq: an arrive orders this thread's earlier memory operations, so the
-      // reductions come after it and the MMA thread never waits on their round trip
-      uint32_t dqv[128];
+      float* dqrow = p.dq + (((long long)b * p.L + (q_valid ? phys_q : 0)) * p.Hq + h) * d + hd0;
+      // this warp's half of the dQ row into registers first, then free the TMEM
+      // columns, then add into dq: an arrive orders this thread's earlier memory
+      // operations, so the reductions come after it and the MMA thread never
+      // waits on their round trip
+      uint32_t dqv[64];
       __syncwarp();
-      ptx::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&dqv[0]));
-      ptx::tmem_ld32(tS + 32u, *reinterpret_cast<uint32_t(*)[32]>(&dqv[32]));
-      if (d == 128) {
-        ptx::tmem_ld32(tS + 64u, *reinterpret_cast<uint32_t(*)[32]>(&dqv[64]));
-        ptx::tmem_ld32(tS + 96u, *reinterpret_cast<uint32_t(*)[32]>(&dqv[96]));
-      }
+      ptx::tmem_ld32(tS + (uint32_t)hd0, *reinterpret_cast<uint32_t(*)[32]>(&dqv[0]));
+      if (d == 128) ptx::tmem_ld32(tS + (uint32_t)hd0 + 32u, *reinterpret_cast<uint32_t(*)[32]>(&dqv[32]));
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(BB_SFREE));
       if (q_valid) {
 #pragma unroll
-        for (int v4 = 0; v4 < 32; ++v4)
-          if (4 * v4 < d)
+        for (int v4 = 0; v4 < 16; ++v4)
+          if (4 * v4 < d / 2)
             red_add_v4(dqrow + 4 * v4, __uint_as_float(dqv[4 * v4]) * p.scale,
                        __uint_as_float(dqv[4 * v4 + 1]) * p.scale, __uint_as_float(dqv[4 * v4 + 2]) * p.scale,
                        __uint_as_float(dqv[4 * v4 + 3]) * p.scale);
       }
     }
     if (ok) {
-      // dK and dV of key tile j, row = key row: the last GRAD commit covers every MMA
+      // dK and dV of key tile j, row = key row, this warp's half of the head dim:
+      // the last GRAD commit covers every MMA
       const int phys_k = b_phys(j * kTile + row, p);
-      for (int c32 = 0; c32 < d / 32; ++c32) {
+      for (int c32 = hd0 / 32; c32 < (hd0 + d / 2) / 32; ++c32) {
         uint32_t kv[32], vv[32];
         __syncwarp();
         ptx::tmem_ld32(tdK + 32u * c32, kv);
@@ -343,10 +344,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
       }
     }
   }
+
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (warp == 5) ptx::tmem_dealloc(tmem, 512);
+  if (warp == 9) ptx::tmem_dealloc(tmem, 512);
 }
 
 // dO = dout sigmoid(g) (input dtype), D = sum_c dout out, dgate = dout out (1 - sigmoid(g)).
