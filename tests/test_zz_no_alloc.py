@@ -91,3 +91,23 @@ def test_noalloc_refuses_shapes_beyond_its_array():
     torch.cuda.synchronize()
     assert rc == _lib.ERR_TOO_LARGE
     assert int(status.item()) == 0
+
+
+def test_noalloc_writes_the_same_lse():
+    case = CASES[1]  # scanline, gated
+    dev = torch.device("cuda:0")
+    q, k, v, g = (t.to(dev) if t is not None else None for t in S.make_inputs(case))
+    want = torch.full((1, case.q_heads, case.seq_len), float("nan"), dtype=torch.float32, device=dev)
+    K.attention(q, k, v, g, text_len=case.text_len, grid_h=case.grid_h, grid_w=case.grid_w, mode=case.mode,
+                window=case.window, tile_aligned=case.tile_aligned, text_pad=case.text_pad, lse=want)
+    got = torch.full_like(want, float("nan"))
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    p = _params(case, q, k, v, g, out, status)
+    p.lse = got.data_ptr()
+    rc = _lib.lib().krea_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), out.data_ptr(),
+                                          case.text_len, case.grid_h, case.grid_w, _lib.MODE[case.mode],
+                                          ctypes.byref(p), torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert rc == 0 and int(status.item()) == 0
+    assert torch.equal(got, want)  # the same kernel on the same inputs: bit for bit
