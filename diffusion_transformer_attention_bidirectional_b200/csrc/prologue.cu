@@ -5,6 +5,9 @@
 //
 //   y = rope(x * gamma / sqrt(mean(x^2) + eps))   per (batch, token, head) vector
 //
+// in fp32 (pairs of channels per packed instruction), the reciprocal square
+// root to within 2^-22 relative, rounded once to the input dtype.
+//
 // rope turns adjacent channel pairs (2i, 2i+1) of three consecutive channel
 // groups (axes_dim[0..2] channels) by pos[t][a] * theta^(-2i / axes_dim[a]).
 // The cos/sin of every (token, pair) come from a table built once per geometry
@@ -20,6 +23,7 @@
 #include <cuda_runtime.h>
 
 #include "krea_internal.h"
+#include "ptx_sm100.cuh"
 
 namespace krea {
 namespace {
@@ -73,9 +77,10 @@ __global__ void __launch_bounds__(512, CODES ? 1 : 2) prologue_kernel(PrologueDe
   const int c0 = 8 * li;            // this lane's channels c0 .. c0 + 7
   const int pj0 = c0 / 2;           // and its rotary pairs pj0 .. pj0 + 3
   __shared__ float red[16];
-  float g[8];
+  uint64_t g2[4];  // the weights as f32 pairs: the arithmetic below is packed (two lanes per op)
 #pragma unroll
-  for (int j = 0; j < 8; ++j) g[j] = p.gamma ? p.gamma[c0 + j] : 1.0f;
+  for (int j = 0; j < 4; ++j)
+    g2[j] = p.gamma ? ptx::f2(p.gamma[c0 + 2 * j], p.gamma[c0 + 2 * j + 1]) : ptx::f2(1.0f, 1.0f);
   float keep[CODES ? STEPS : 1][8];  // stored values, for the codes
   float amax = 0.f;
   uint4 raw[STEPS];  // every load of the thread is issued before the first use
@@ -90,38 +95,45 @@ __global__ void __launch_bounds__(512, CODES ? 1 : 2) prologue_kernel(PrologueDe
   for (int st = 0; st < STEPS; ++st) {
     const int t = blk * kTile + warp * 8 + st * RPW + sub;
     const bool live = t < p.L;
-    float x[8];
+    uint64_t x2[4];  // channel pairs (2j, 2j+1) of this lane, as f32 pairs
     float ss = 0.f;
-    if (live) {
-      const uint4 u = raw[st];
+    {
+      const uint4 u = raw[st];  // zero for rows past L
       const uint16_t* e = reinterpret_cast<const uint16_t*>(&u);
+      uint64_t acc = ptx::f2(0.f, 0.f);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        x[j] = ld_f<BF16>(e[j]);
-        ss = __fmaf_rn(x[j], x[j], ss);
+      for (int j = 0; j < 4; ++j) {
+        x2[j] = ptx::f2(ld_f<BF16>(e[2 * j]), ld_f<BF16>(e[2 * j + 1]));
+        acc = ptx::fma2(x2[j], x2[j], acc);
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) x[j] = 0.f;
+      float s0, s1;
+      ptx::unf2(acc, s0, s1);
+      ss = s0 + s1;
     }
 #pragma unroll
     for (int o = LPR / 2; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
     if (live) {
-      // 1 / sqrt(mean + eps), each step rounded once (IEEE)
-      const float r = __frsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)D), p.eps));
+      // 1 / sqrt(mean + eps): 1/D is a power of two (exact), rsqrt to within 2^-22
+      const float r = rsqrtf(__fadd_rn(ss * (1.0f / (float)D), p.eps));
+      const uint64_t r2 = ptx::f2(r, r);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(__fmul_rn(x[j], r), g[j]);
+      for (int j = 0; j < 4; ++j) x2[j] = ptx::mul2(ptx::mul2(x2[j], r2), g2[j]);
       const float4* tab = reinterpret_cast<const float4*>(p.table + 2LL * ((long long)t * p.n_pairs + pj0));
 #pragma unroll
       for (int q2 = 0; q2 < 2; ++q2) {  // two pairs per 16-byte table load
         if (pj0 + 2 * q2 >= p.n_pairs) break;
         const float4 cs = tab[q2];
-        const float a0 = x[4 * q2], a1 = x[4 * q2 + 1], b0 = x[4 * q2 + 2], b1 = x[4 * q2 + 3];
-        x[4 * q2] = __fmaf_rn(a0, cs.x, -__fmul_rn(a1, cs.y));
-        x[4 * q2 + 1] = __fmaf_rn(a0, cs.y, __fmul_rn(a1, cs.x));
-        x[4 * q2 + 2] = __fmaf_rn(b0, cs.z, -__fmul_rn(b1, cs.w));
-        x[4 * q2 + 3] = __fmaf_rn(b0, cs.w, __fmul_rn(b1, cs.z));
+        // (a0, a1) -> (a0 c - a1 s, a0 s + a1 c) = (a0, a0) (c, s) + (a1, a1) (-s, c)
+        float a0, a1, b0, b1;
+        ptx::unf2(x2[2 * q2], a0, a1);
+        ptx::unf2(x2[2 * q2 + 1], b0, b1);
+        x2[2 * q2] = ptx::fma2(ptx::f2(a1, a1), ptx::f2(-cs.y, cs.x), ptx::mul2(ptx::f2(a0, a0), ptx::f2(cs.x, cs.y)));
+        x2[2 * q2 + 1] =
+            ptx::fma2(ptx::f2(b1, b1), ptx::f2(-cs.w, cs.z), ptx::mul2(ptx::f2(b0, b0), ptx::f2(cs.z, cs.w)));
       }
+      float x[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) ptx::unf2(x2[j], x[2 * j], x[2 * j + 1]);
       uint4 u;
       uint16_t* e = reinterpret_cast<uint16_t*>(&u);
 #pragma unroll
