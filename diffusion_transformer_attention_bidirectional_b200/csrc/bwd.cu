@@ -44,7 +44,8 @@ namespace {
 constexpr int kBThreads = 320;
 constexpr uint32_t kBBox = 16384;        // 128 rows x 128 bytes
 constexpr uint32_t BS_K = 0, BS_V = 32768, BS_Q = 65536, BS_DO = 98304, BS_P = 131072, BS_DS = 163840;
-constexpr uint32_t BS_BAR = 196608;
+constexpr uint32_t BS_RED = 196608;   // 8 warps x 4 KB: dQ rows turned so a reduction covers whole rows
+constexpr uint32_t BS_BAR = BS_RED + 8 * 4096;
 enum { BB_KV = 0, BB_QF, BB_SDP, BB_PDS, BB_GRAD, BB_SFREE, BB_DRAIN, BB_QFREE, BB_N };
 constexpr uint32_t BS_TMEM = BS_BAR + 8 * BB_N;
 constexpr uint32_t BS_ABORT = BS_TMEM + 4;
@@ -297,7 +298,6 @@ __global__ void __launch_bounds__(kBThreads, 1)
       ok = b_wait_warp(ctl, bar(BB_GRAD), s & 1);
       if (!ok) break;
       ptx::tc_fence_after();
-      float* dqrow = p.dq + (((long long)b * p.L + (q_valid ? phys_q : 0)) * p.Hq + h) * d + hd0;
       // this warp's half of the dQ row into registers first, then free the TMEM
       // columns, then add into dq: an arrive orders this thread's earlier memory
       // operations, so the reductions come after it and the MMA thread never
@@ -310,13 +310,35 @@ __global__ void __launch_bounds__(kBThreads, 1)
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(BB_SFREE));
-      if (q_valid) {
+      // Thread = row holds 32 consecutive floats per round; the warp's 32 x 32 block
+      // goes through a 4 KB swizzled scratch so that each reduction instruction
+      // covers 4 rows x 128 contiguous bytes (whole sectors) instead of 32 rows x
+      // 16 bytes: half the L2 atomic operations.
+      uint8_t* scr = sb + BS_RED + (uint32_t)warp * 4096u;
+      const uint32_t wsw = (uint32_t)(lane & 7);
+      const int rsub = lane >> 3, piece = lane & 7;  // read side: row 4 i + rsub, 16-byte piece
 #pragma unroll
-        for (int v4 = 0; v4 < 16; ++v4)
-          if (4 * v4 < d / 2)
-            red_add_v4(dqrow + 4 * v4, __uint_as_float(dqv[4 * v4]) * p.scale,
-                       __uint_as_float(dqv[4 * v4 + 1]) * p.scale, __uint_as_float(dqv[4 * v4 + 2]) * p.scale,
-                       __uint_as_float(dqv[4 * v4 + 3]) * p.scale);
+      for (int rnd = 0; rnd < 2; ++rnd) {  // 32 floats of the row per round (registers: constant trip)
+        if (rnd >= d / 64) break;
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4*>(scr + (uint32_t)lane * 128u + (((uint32_t)k ^ wsw) << 4)) =
+              make_uint4(dqv[32 * rnd + 4 * k], dqv[32 * rnd + 4 * k + 1], dqv[32 * rnd + 4 * k + 2],
+                         dqv[32 * rnd + 4 * k + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + rsub;  // row within the warp (its thread is lane rr)
+          const int pq = __shfl_sync(0xffffffffu, phys_q, rr);
+          if (pq >= 0) {
+            const uint4 u = *reinterpret_cast<const uint4*>(scr + (uint32_t)rr * 128u +
+                                                           (((uint32_t)piece ^ (uint32_t)(rr & 7)) << 4));
+            float* dst = p.dq + (((long long)b * p.L + pq) * p.Hq + h) * d + hd0 + 32 * rnd + 4 * piece;
+            red_add_v4(dst, __uint_as_float(u.x) * p.scale, __uint_as_float(u.y) * p.scale,
+                       __uint_as_float(u.z) * p.scale, __uint_as_float(u.w) * p.scale);
+          }
+        }
       }
     }
     if (ok) {
