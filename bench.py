@@ -618,7 +618,7 @@ def main():
     try:
         res = run_ours(args, rank, world, device)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            rows = 64
+            rows = 192  # about 10 s of fp64 work on a 16-core host
             f, t = oracle_sample(rows)
             res["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
                                    "kind": "oracle",
