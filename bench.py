@@ -240,6 +240,59 @@ def time_prologue(K, device, stream, flush, P, reps: int = 8):
             "bound": "hbm", "peak_source": f"{P['source']} copy bandwidth", "l2": "flushed before each pass"}
 
 
+def time_exchange(K, device, stream, flush, P, world: int = 4, reps: int = 8):
+    """The sequence <-> head exchange at the 4 MP shape with `world` ranks emulated
+    on this GPU (every destination in its own HBM): q through the QK prologue
+    into the head shards, gate copied into them, the fp32 output copied back to
+    the token shards. Bound by HBM here (by NVLink on real peers); algorithmic
+    bytes = every row read once and written once."""
+    from diffusion_transformer_attention_bidirectional_b200 import seqpar
+    from synth import inputs as S
+
+    pc = S.Case("exchange_4mp", 1, 48, 12, 128, 512, 128, 128, dtype="bf16", mode="dense", seed=93, gate=True,
+                prologue=True)
+    q_raw, _, _, g = S.make_inputs(pc)
+    qd, gd = q_raw.to(device), g.to(device)
+    B, L, Hq, d = qd.shape
+    Ls = L // world
+    table = K.rope_table(K.rope_positions(pc.text_len, pc.grid_h, pc.grid_w, device))
+    qh = [torch.empty(B, L, Hq // world, d, dtype=qd.dtype, device=device) for _ in range(world)]
+    gh = [torch.empty_like(x) for x in qh]
+    oh = [torch.empty(B, L, Hq // world, d, dtype=torch.float32, device=device) for _ in range(world)]
+    os_ = [torch.empty(B, Ls, Hq, d, dtype=torch.float32, device=device) for _ in range(world)]
+    dq, dg, do = seqpar.Destinations.of(qh), seqpar.Destinations.of(gh), seqpar.Destinations.of(os_)
+
+    def timed(fn):
+        times = []
+        for it in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for r in range(world):
+                fn(r)
+            b.record(stream)
+            torch.cuda.synchronize(device)
+            if it >= 3:
+                times.append(a.elapsed_time(b))
+        return sorted(times)[len(times) // 2]
+
+    res = {"world_emulated": world, "peak_gbs": P["hbm_gbs"], "bound": "hbm",
+           "peak_source": f"{P['source']} copy bandwidth", "l2": "flushed before each pass"}
+    legs = {
+        "qk_prologue_to_heads": (lambda r: seqpar.qk_prologue_to_heads(qd[:, r * Ls:(r + 1) * Ls], table, dq, r),
+                                 2 * qd.numel() * qd.element_size()),
+        "seq_to_heads(gate)": (lambda r: seqpar.seq_to_heads(gd[:, r * Ls:(r + 1) * Ls], dg, r),
+                               2 * gd.numel() * gd.element_size()),
+        "heads_to_seq(out fp32)": (lambda r: seqpar.heads_to_seq(oh[r], do, r), 2 * B * L * Hq * d * 4),
+    }
+    for name, (fn, nbytes) in legs.items():
+        ms = timed(fn)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 4), "algorithmic_bytes": nbytes, "achieved_gbs": round(gbs, 1),
+                     "frac": round(gbs / P["hbm_gbs"], 4)}
+    return res
+
+
 def time_backward(K, device, stream, flush, P, reps: int = 6):
     """The backward (prep + dq/dk/dv kernel) on the dense 1 MP shape: 48/12 heads,
     d 128, bf16, gate. Algorithmic FLOPs: five products of 2 d per admitted pair
@@ -579,6 +632,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prologue-only", action="store_true",
                     help="time only the QK prologue at the 4 MP shape (profiling)")
+    ap.add_argument("--exchange-only", action="store_true",
+                    help="time only the sequence <-> head exchange (ranks emulated on one GPU)")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only the backward at the dense 1 MP shape (profiling)")
     ap.add_argument("--no-comparisons", action="store_true",
@@ -607,12 +662,12 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
-    if args.prologue_only or args.backward_only:
+    if args.prologue_only or args.backward_only or args.exchange_only:
         import diffusion_transformer_attention_bidirectional_b200 as K
 
         torch.cuda.set_device(device)
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
-        fn = time_prologue if args.prologue_only else time_backward
+        fn = time_prologue if args.prologue_only else time_exchange if args.exchange_only else time_backward
         print(json.dumps(fn(K, device, torch.cuda.current_stream(device), flush, peaks())), flush=True)
         return
     try:

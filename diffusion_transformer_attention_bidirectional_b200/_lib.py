@@ -73,6 +73,23 @@ class RopeParams(ctypes.Structure):
     _fields_ = [("axes_dim", ctypes.c_int32 * 3), ("theta", ctypes.c_float), ("eps", ctypes.c_float)]
 
 
+EXCHANGE_MAX_RANKS = 16
+IPC_HANDLE_BYTES = 64
+
+
+class Exchange(ctypes.Structure):
+    """krea_exchange_t."""
+
+    _fields_ = [
+        ("world", ctypes.c_int32),
+        ("rank", ctypes.c_int32),
+        ("tokens_per_rank", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("dst", ctypes.c_void_p * EXCHANGE_MAX_RANKS),
+        ("dst_stride", ctypes.c_int64 * 3),
+    ]
+
+
 class WsLayout(ctypes.Structure):
     """krea_attn_ws_layout_t."""
 
@@ -100,6 +117,16 @@ SIGNATURES = {
     "krea_attn_rope_table": (_I, [_VP, _I, ctypes.POINTER(RopeParams), _VP, _VP]),
     "krea_attn_qk_prologue": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int64),
                                    ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(RopeParams), _VP, _VP, _VP]),
+    "krea_attn_seq_to_heads": (_I, [_VP, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int64),
+                                    ctypes.POINTER(Exchange), _VP]),
+    "krea_attn_heads_to_seq": (_I, [_VP, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int64),
+                                    ctypes.POINTER(Exchange), _VP]),
+    "krea_attn_qk_prologue_to_heads": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int64),
+                                            ctypes.POINTER(RopeParams), ctypes.POINTER(Exchange), _VP]),
+    "krea_attn_ipc_alloc": (_I, [ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p), _VP]),
+    "krea_attn_ipc_free": (_I, [_VP]),
+    "krea_attn_ipc_open": (_I, [_VP, ctypes.POINTER(ctypes.c_void_p)]),
+    "krea_attn_ipc_close": (_I, [_VP]),
     "krea_attn_clear_cache": (None, []),
     "krea_attn_error_string": (ctypes.c_char_p, [_I]),
     "krea_attn_abi_version": (_I, []),

@@ -12,7 +12,7 @@ CSRC = PKG / "csrc"
 LIB = PKG / "libkrea_attn.so"
 BUILD_DIR = PKG.parent / "_build"
 
-SOURCES = ["api.cpp", "tilemap.cpp", "mapgen.cu", "prologue.cu", "quant.cu", "attn_sm100.cu", "bwd.cu", "noalloc.cu"]
+SOURCES = ["api.cpp", "tilemap.cpp", "mapgen.cu", "prologue.cu", "quant.cu", "attn_sm100.cu", "bwd.cu", "noalloc.cu", "exchange.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "-I", str(PKG.parent / "include")]

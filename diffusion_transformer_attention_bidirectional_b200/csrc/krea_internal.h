@@ -61,7 +61,28 @@ struct PrologueDevParams {
   long long y_stride[3];
   int B, L, H, d, nt, n_pairs;
   float eps;
+  // Store into another rank's buffer: when heads_per_peer > 0, head h of token t
+  // goes to y_peer[h / heads_per_peer] at head h % heads_per_peer and token
+  // t + token_offset (y is unused); token_offset also selects the table row.
+  void* y_peer[KREA_EXCHANGE_MAX_RANKS];
+  int heads_per_peer;
+  int token_offset;
 };
+
+// Sequence <-> head exchange (exchange.cu): a strided copy of rows of `chunks`
+// 16-byte pieces from src [B, Ls, Hs] into dst[peer] by the rule of
+// krea_attn_seq_to_heads (to_heads) or krea_attn_heads_to_seq.
+struct ExchangeDevParams {
+  const void* src;
+  void* dst[KREA_EXCHANGE_MAX_RANKS];
+  long long s_stride[3], d_stride[3];  // elements
+  int B, Ls, Hs;
+  int chunk_shift;  // log2 of the 16-byte pieces per row
+  int es;           // element bytes
+  int to_heads;
+  int rank, tokens_per_rank, heads_per_rank;
+};
+int launch_exchange(const ExchangeDevParams& p, void* stream);
 int launch_rope_table(const int32_t* pos, int tokens, const int axes[3], double theta, float* table, void* stream);
 int launch_prologue(const PrologueDevParams& p, bool bf16, void* stream);
 

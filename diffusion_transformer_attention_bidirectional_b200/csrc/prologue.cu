@@ -77,6 +77,14 @@ __global__ void __launch_bounds__(512, CODES ? 1 : 2) prologue_kernel(PrologueDe
   const int c0 = 8 * li;            // this lane's channels c0 .. c0 + 7
   const int pj0 = c0 / 2;           // and its rotary pairs pj0 .. pj0 + 3
   __shared__ float red[16];
+  // where this head's rows go: y, or a peer's buffer of the sequence <-> head exchange
+  uint16_t* ybase = static_cast<uint16_t*>(p.y);
+  int hy = h;
+  if (p.heads_per_peer > 0) {
+    const int j = h / p.heads_per_peer;
+    ybase = static_cast<uint16_t*>(p.y_peer[j]);
+    hy = h - j * p.heads_per_peer;
+  }
   uint64_t g2[4];  // the weights as f32 pairs: the arithmetic below is packed (two lanes per op)
 #pragma unroll
   for (int j = 0; j < 4; ++j)
@@ -118,7 +126,8 @@ __global__ void __launch_bounds__(512, CODES ? 1 : 2) prologue_kernel(PrologueDe
       const uint64_t r2 = ptx::f2(r, r);
 #pragma unroll
       for (int j = 0; j < 4; ++j) x2[j] = ptx::mul2(ptx::mul2(x2[j], r2), g2[j]);
-      const float4* tab = reinterpret_cast<const float4*>(p.table + 2LL * ((long long)t * p.n_pairs + pj0));
+      const long long tg = (long long)t + p.token_offset;  // token in the whole sequence
+      const float4* tab = reinterpret_cast<const float4*>(p.table + 2LL * (tg * p.n_pairs + pj0));
 #pragma unroll
       for (int q2 = 0; q2 < 2; ++q2) {  // two pairs per 16-byte table load
         if (pj0 + 2 * q2 >= p.n_pairs) break;
@@ -144,8 +153,7 @@ __global__ void __launch_bounds__(512, CODES ? 1 : 2) prologue_kernel(PrologueDe
           amax = fmaxf(amax, fabsf(keep[st][j]));
         }
       }
-      *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.y) + b * p.y_stride[0] + (long long)t * p.y_stride[1] +
-                                h * p.y_stride[2] + c0) = u;
+      *reinterpret_cast<uint4*>(ybase + b * p.y_stride[0] + tg * p.y_stride[1] + hy * p.y_stride[2] + c0) = u;
     } else if constexpr (CODES) {
 #pragma unroll
       for (int j = 0; j < 8; ++j) keep[st][j] = 0.f;

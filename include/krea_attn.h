@@ -78,7 +78,7 @@ typedef enum {
   KREA_ERR_DEVICE_TIMEOUT = -5,  /* written to *status: a bounded wait in a kernel ran out */
   KREA_ERR_DEVICE_BOUNDS = -6,   /* written to *status: a kernel met an out-of-range index */
   KREA_ERR_NO_DEVICE = -7,       /* no CUDA device, or not an sm_100 device */
-  KREA_ERR_TOO_LARGE = -8        /* krea_attn_fwd_noalloc: the shape needs more scratch than its fixed array */
+  KREA_ERR_TOO_LARGE = -8        /* a fixed limit of the call: krea_attn_fwd_noalloc's scratch, the exchange's size */
 } krea_status_t;
 
 /* Kind bits of one tile of a map (krea_attn_get_map). */
@@ -215,6 +215,76 @@ KREA_API int krea_attn_qk_prologue(const void* x, void* y, const float* gamma, c
                                    int tokens, int heads, int head_dim, int dtype, const int64_t* x_stride,
                                    const int64_t* y_stride, const krea_rope_params_t* rope, int8_t* codes,
                                    float* scales, void* stream);
+
+/* ---- sequence <-> head exchange (sequence-parallel callers) ----------------
+ * A caller whose block holds the joint [text, image] sequence split by token
+ * across `world` ranks (rank r: tokens [r * tokens_per_rank, (r + 1) *
+ * tokens_per_rank)) turns it into a split by head before the attention core and
+ * back after it. Every head of the core is independent, and query head h reads
+ * kv head h / (Hq / Hkv) ("Krea 2 TileMix Attention (FP16/INT8 tiles)", section
+ * "What it actually patches": the key/value heads are repeated to the query
+ * heads), so rank j can run the ordinary call on query heads [j Hq / world,
+ * (j + 1) Hq / world) and kv heads [j Hkv / world, (j + 1) Hkv / world) over the
+ * whole sequence. The pages describe no multi-GPU split; this is the plain one.
+ *
+ * The exchange is a push: each rank stores its rows straight into the
+ * destination buffers of every rank (peer memory over NVLink, or this device's
+ * own memory), with no packing pass and no library collective. The caller
+ * orders the ranks around it: no rank may read a destination before every rank's
+ * exchange into it has completed (a stream-ordered barrier, e.g. a one-element
+ * all-reduce), and no rank may overwrite a destination that its owner still
+ * reads. */
+#define KREA_EXCHANGE_MAX_RANKS 16
+typedef struct {
+  int32_t world;            /* ranks sharing the sequence, 1 .. KREA_EXCHANGE_MAX_RANKS */
+  int32_t rank;             /* this rank, 0 .. world - 1 */
+  int32_t tokens_per_rank;  /* tokens of every shard (> 0); the sequence holds world * tokens_per_rank */
+  int32_t reserved;         /* 0 */
+  void* dst[KREA_EXCHANGE_MAX_RANKS]; /* dst[j]: rank j's destination buffer as this process addresses it
+                                         (device memory of this GPU or an opened IPC mapping of a peer's);
+                                         16-byte aligned; entries past world are ignored */
+  int64_t dst_stride[3];    /* element strides (b, token, head) shared by every dst[j]; multiples of 16 bytes */
+} krea_exchange_t;
+
+/* Token shard -> head shards. x: this rank's rows [batch, tokens_per_rank, heads,
+ * head_dim] (device, strides x_stride over (b, token, head), head_dim contiguous).
+ * heads % world == 0; row (b, t, h) is copied unchanged to dst[h / (heads /
+ * world)] at (b, rank * tokens_per_rank + t, h mod (heads / world)). dtype
+ * KREA_F16, KREA_BF16 or KREA_F32; head_dim 64 or 128. One batch entry of x
+ * holds fewer than 2^35 bytes (KREA_ERR_TOO_LARGE otherwise). */
+KREA_API int krea_attn_seq_to_heads(const void* x, int batch, int heads, int head_dim, int dtype,
+                                    const int64_t* x_stride, const krea_exchange_t* ex, void* stream);
+
+/* Head shard -> token shards, the inverse. y: this rank's heads over the whole
+ * sequence [batch, world * tokens_per_rank, heads, head_dim]; row (b, t, h) goes
+ * to dst[t / tokens_per_rank] at (b, t mod tokens_per_rank, rank * heads + h).
+ * Same types and limits as krea_attn_seq_to_heads. */
+KREA_API int krea_attn_heads_to_seq(const void* y, int batch, int heads, int head_dim, int dtype,
+                                    const int64_t* y_stride, const krea_exchange_t* ex, void* stream);
+
+/* The QK prologue of krea_attn_qk_prologue on this rank's token shard x [batch,
+ * tokens_per_rank, heads, head_dim], its output stored as krea_attn_seq_to_heads
+ * stores rows: y of row (b, t, h) lands in dst[h / (heads / world)] at (b, rank *
+ * tokens_per_rank + t, h mod (heads / world)). The rotation of row t uses table
+ * row rank * tokens_per_rank + t: the table covers the whole sequence. dtype
+ * KREA_F16 or KREA_BF16; no INT8 codes in this form. */
+KREA_API int krea_attn_qk_prologue_to_heads(const void* x, const float* gamma, const float* table, int batch,
+                                            int heads, int head_dim, int dtype, const int64_t* x_stride,
+                                            const krea_rope_params_t* rope, const krea_exchange_t* ex,
+                                            void* stream);
+
+/* Destination buffers other processes can map (CUDA IPC on one node).
+ * krea_attn_ipc_alloc allocates `bytes` of device memory on the current device
+ * (a dedicated allocation: the handle maps exactly this buffer) and writes its
+ * handle (KREA_IPC_HANDLE_BYTES opaque bytes) to `handle`; krea_attn_ipc_free
+ * releases it. krea_attn_ipc_open maps another process's handle into this one
+ * (not one of this process's own allocations) and krea_attn_ipc_close unmaps
+ * it. Failures return KREA_ERR_CUDA with nothing allocated or mapped. */
+#define KREA_IPC_HANDLE_BYTES 64
+KREA_API int krea_attn_ipc_alloc(size_t bytes, void** ptr, void* handle);
+KREA_API int krea_attn_ipc_free(void* ptr);
+KREA_API int krea_attn_ipc_open(const void* handle, void** ptr);
+KREA_API int krea_attn_ipc_close(void* ptr);
 
 /* Run only the TileMix quantiser (key mean, centred keys, INT8 codes and scales)
  * into params->workspace, laid out as krea_attn_workspace_layout() says. */

@@ -133,3 +133,68 @@ def test_prologue_arguments_rejected_without_gpu():
 def test_rope_positions_layout():
     pos = K.rope_positions(2, 2, 3)
     assert pos.tolist() == [[0, 0, 0], [1, 0, 0], [0, 0, 0], [0, 0, 1], [0, 0, 2], [0, 1, 0], [0, 1, 1], [0, 1, 2]]
+
+
+def test_exchange_layout_matches_header():
+    fields = [f for f, _ in _lib.Exchange._fields_]
+    prog = "#include <stdio.h>\n#include <stddef.h>\n#include \"krea_attn.h\"\nint main(void){\n"
+    prog += 'printf("%zu\\n", sizeof(krea_exchange_t));\n'
+    for f in fields:
+        prog += f'printf("%zu\\n", offsetof(krea_exchange_t, {f}));\n'
+    prog += 'printf("%d %d\\n", KREA_EXCHANGE_MAX_RANKS, KREA_IPC_HANDLE_BYTES);\nreturn 0;}\n'
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(prog)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True).stdout.split()]
+    assert vals[0] == ctypes.sizeof(_lib.Exchange)
+    for f, off in zip(fields, vals[1:]):
+        assert getattr(_lib.Exchange, f).offset == off, f
+    assert vals[-2:] == [_lib.EXCHANGE_MAX_RANKS, _lib.IPC_HANDLE_BYTES]
+
+
+def test_exchange_arguments_rejected_without_gpu():
+    L = _lib.lib()
+    ptr = 1 << 20
+    s = (ctypes.c_int64 * 3)(1 << 20, 1024, 128)
+
+    def ex(world=2, rank=0, tokens=64, reserved=0, dst_ok=True):
+        e = _lib.Exchange()
+        e.world, e.rank, e.tokens_per_rank, e.reserved = world, rank, tokens, reserved
+        for j in range(max(0, min(world, 16))):
+            e.dst[j] = ptr if dst_ok else None
+        for i in range(3):
+            e.dst_stride[i] = s[i]
+        return e
+
+    def s2h(e, heads=8, d=128, dtype=1, x=ptr):
+        return L.krea_attn_seq_to_heads(x, 1, heads, d, dtype, s, ctypes.byref(e), None)
+
+    assert s2h(ex()) == _lib.ERR_NO_DEVICE                    # well-formed: only the device is missing
+    assert s2h(ex(), d=96) == _lib.ERR_UNSUPPORTED
+    assert s2h(ex(), dtype=7) == _lib.ERR_INVALID_ARG
+    assert s2h(ex(world=0)) == _lib.ERR_INVALID_ARG
+    assert s2h(ex(world=17)) == _lib.ERR_INVALID_ARG
+    assert s2h(ex(rank=2)) == _lib.ERR_INVALID_ARG
+    assert s2h(ex(tokens=0)) == _lib.ERR_INVALID_ARG
+    assert s2h(ex(reserved=1)) == _lib.ERR_INVALID_ARG
+    assert s2h(ex(dst_ok=False)) == _lib.ERR_INVALID_ARG
+    assert s2h(ex(world=3), heads=8) == _lib.ERR_INVALID_ARG  # 8 heads do not split over 3 ranks
+    assert s2h(ex(), x=ptr + 8) == _lib.ERR_INVALID_ARG       # misaligned rows
+    assert s2h(ex(tokens=1 << 24), heads=64) == _lib.ERR_TOO_LARGE
+    # the inverse direction takes any head count (this rank's heads)
+    assert L.krea_attn_heads_to_seq(ptr, 1, 3, 128, 1, s, ctypes.byref(ex(world=3)), None) == _lib.ERR_NO_DEVICE
+    r = K.rope_params(128)
+    pro = L.krea_attn_qk_prologue_to_heads
+    assert pro(ptr, None, ptr, 1, 8, 128, 1, s, ctypes.byref(r), ctypes.byref(ex()), None) == _lib.ERR_NO_DEVICE
+    assert pro(ptr, None, ptr, 1, 8, 128, 2, s, ctypes.byref(r), ctypes.byref(ex()), None) == _lib.ERR_UNSUPPORTED
+    assert pro(ptr, None, ptr, 1, 6, 128, 1, s, ctypes.byref(r), ctypes.byref(ex(world=4)),
+               None) == _lib.ERR_INVALID_ARG
+    p = ctypes.c_void_p()
+    h = (ctypes.c_ubyte * _lib.IPC_HANDLE_BYTES)()
+    assert L.krea_attn_ipc_alloc(0, ctypes.byref(p), h) == _lib.ERR_INVALID_ARG
+    assert L.krea_attn_ipc_alloc(256, ctypes.byref(p), h) == _lib.ERR_NO_DEVICE
+    assert L.krea_attn_ipc_open(h, ctypes.byref(p)) == _lib.ERR_NO_DEVICE
+    assert L.krea_attn_ipc_free(None) == _lib.ERR_INVALID_ARG
+    assert L.krea_attn_ipc_close(None) == _lib.ERR_INVALID_ARG

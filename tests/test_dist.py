@@ -71,3 +71,80 @@ def test_partition_covers_units_once():
             assert covered == list(range(Hkv))
             sizes = [b - a for a, b in parts]
             assert max(sizes) - min(sizes) <= 1
+
+
+def _sequence_parallel_worker(rank, world, port, results):
+    """Rank `rank` of a block split by token: the QK prologue on its token shard,
+    an all-to-all to the head split (token order of the shards, heads
+    head_range(.., world, j) to rank j), the oracle core on its heads over the
+    whole sequence, the inverse all-to-all, all in fp64."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import dataclasses
+
+        import numpy as np
+
+        from diffusion_transformer_attention_bidirectional_b200 import seqpar
+        from oracle import krea_oracle as ko
+        from synth import inputs as S
+
+        case = S.Case("seqpar", 1, 4, 2, 64, 16, 8, 8, dtype="f16", mode="scanline", window=3, gate=True,
+                      prologue=True, seed=7)
+        L, Ls = case.seq_len, case.seq_len // world
+        q, k, v, g = S.make_inputs(case)
+        pos = ko.rope_positions(case.text_len, case.grid_h, case.grid_w)
+        t0, t1 = seqpar.token_range(Ls, rank)
+        mine = {"q": torch.from_numpy(ko.qk_prologue(q[:, t0:t1], pos[t0:t1])),
+                "k": torch.from_numpy(ko.qk_prologue(k[:, t0:t1], pos[t0:t1])),
+                "v": v[:, t0:t1].double(), "g": g[:, t0:t1].double()}
+
+        def to_heads(x):  # [1, Ls, H, d] token shard -> [1, L, H / world, d] head shard
+            H = x.shape[2]
+            send = torch.stack([x[:, :, slice(*seqpar.head_range(H, world, j))] for j in range(world)]).contiguous()
+            recv = torch.empty_like(send)
+            dist.all_to_all_single(recv, send)
+            return torch.cat(list(recv), dim=1)  # source ranks hold consecutive token ranges
+
+        def to_seq(y):  # [1, L, Hr, d] head shard -> [1, Ls, world * Hr, d] token shard
+            send = torch.stack([y[:, slice(*seqpar.token_range(Ls, j))] for j in range(world)]).contiguous()
+            recv = torch.empty_like(send)
+            dist.all_to_all_single(recv, send)
+            return torch.cat(list(recv), dim=2)  # source rank j held heads head_range(.., j)
+
+        h = {n: to_heads(x) for n, x in mine.items()}
+        sub = dataclasses.replace(case, q_heads=case.q_heads // world, kv_heads=case.kv_heads // world)
+        o_heads = torch.from_numpy(ko.attention(sub, h["q"], h["k"], h["v"], h["g"])["out"])
+        o_mine = to_seq(o_heads).numpy()
+        full = ko.attention(case, ko.qk_prologue(q, pos), ko.qk_prologue(k, pos), v, g)["out"]
+        results[rank] = float(np.abs(o_mine - full[:, t0:t1]).max())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sequence_parallel_split_reassembles_the_core():
+    world = 2
+    mgr = mp.Manager()
+    results = mgr.dict()
+    mp.spawn(_sequence_parallel_worker, args=(world, _free_port(), results), nprocs=world, join=True)
+    for r in range(world):
+        assert results[r] < 1e-12, results[r]
+
+
+def test_sequence_parallel_ranges():
+    from diffusion_transformer_attention_bidirectional_b200 import seqpar
+
+    assert [seqpar.head_range(48, 4, j) for j in range(4)] == [(0, 12), (12, 24), (24, 36), (36, 48)]
+    assert [seqpar.head_range(12, 4, j) for j in range(4)] == [(0, 3), (3, 6), (6, 9), (9, 12)]
+    # query head h reads kv head h // 4, and both land on the same rank
+    for W in (1, 2, 3, 4, 6, 12):
+        for h in range(48):
+            j = next(r for r in range(W) if seqpar.head_range(48, W, r)[0] <= h < seqpar.head_range(48, W, r)[1])
+            a, b = seqpar.head_range(12, W, j)
+            assert a <= h // 4 < b
+    assert seqpar.token_range(1152, 3) == (3456, 4608)
+    import pytest
+
+    with pytest.raises(ValueError):
+        seqpar.head_range(12, 5, 0)
