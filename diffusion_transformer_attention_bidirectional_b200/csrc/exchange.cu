@@ -18,69 +18,108 @@
 namespace krea {
 namespace {
 
-// Grid (x, B). Batch b's rows (t, h) in source order, 2^chunk_shift pieces of 16
-// bytes each, are numbered i = ((t * Hs + h) << chunk_shift) + piece; thread i
-// of a grid-stride loop moves piece i, four pieces (one grid stride apart) per
-// iteration with the loads issued before the stores. Consecutive threads read
-// consecutive source bytes, and a destination row stays contiguous.
+// Grid (x, B), 256 threads. The rows (t, h) of batch b, in source order, are
+// cut into contiguous runs of rows_per_cta rows, one run per CTA. Each row is
+// 2^SHIFT pieces of 16 bytes: thread `piece` = tid mod 2^SHIFT of row `sub` =
+// tid / 2^SHIFT, so one step of the CTA moves R = 256 / 2^SHIFT whole rows and a
+// warp access covers whole contiguous rows of the source. U steps are in flight
+// (loads first, then stores). The token, head and destination of the thread's
+// row advance by R rows per step without a division.
+template <int SHIFT>
 __global__ void __launch_bounds__(256) exchange_kernel(ExchangeDevParams p) {
+  constexpr int CH = 1 << SHIFT;
+  constexpr int R = 256 / CH;
   constexpr int U = 4;
   const int b = blockIdx.y;
-  const unsigned n = ((unsigned)p.Ls * (unsigned)p.Hs) << p.chunk_shift;
-  const unsigned stride = gridDim.x * blockDim.x;
-  const unsigned mask = (1u << p.chunk_shift) - 1u;
-  const char* src = static_cast<const char*>(p.src) + (long long)b * p.s_stride[0] * p.es;
-  for (unsigned base = blockIdx.x * blockDim.x + threadIdx.x; base < n; base += U * stride) {
-    uint4 v[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const unsigned i = base + u * stride;
-      if (i < n) {
-        const unsigned row = i >> p.chunk_shift;
-        const unsigned t = row / (unsigned)p.Hs, h = row - t * (unsigned)p.Hs;
-        v[u] = __ldg(reinterpret_cast<const uint4*>(src + ((long long)t * p.s_stride[1] + (long long)h * p.s_stride[2]) * p.es +
-                                                    16u * (i & mask)));
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const unsigned i = base + u * stride;
-      if (i < n) {
-        const unsigned row = i >> p.chunk_shift;
-        const int t = (int)(row / (unsigned)p.Hs), h = (int)(row - (unsigned)t * (unsigned)p.Hs);
-        int peer, td, hd;
-        if (p.to_heads) {
-          peer = h / p.heads_per_rank;
-          hd = h - peer * p.heads_per_rank;
-          td = p.rank * p.tokens_per_rank + t;
-        } else {
-          peer = t / p.tokens_per_rank;
-          td = t - peer * p.tokens_per_rank;
-          hd = p.rank * p.Hs + h;
-        }
-        char* dst = static_cast<char*>(p.dst[peer]);
-        *reinterpret_cast<uint4*>(dst + ((long long)b * p.d_stride[0] + (long long)td * p.d_stride[1] +
-                                         (long long)hd * p.d_stride[2]) * p.es + 16u * (i & mask)) = v[u];
-      }
-    }
+  const int piece = threadIdx.x & (CH - 1);
+  const int sub = threadIdx.x >> SHIFT;
+  const long long rows = (long long)p.Ls * p.Hs;
+  const long long r0 = (long long)blockIdx.x * p.rows_per_cta;
+  const long long r1 = r0 + p.rows_per_cta < rows ? r0 + p.rows_per_cta : rows;
+  long long row = r0 + sub;
+  if (row >= r1) return;
+  const int dt = R / p.Hs, dh = R % p.Hs;  // one step: R rows = dt tokens + dh heads
+  int t = (int)(row / p.Hs), h = (int)(row - (long long)t * p.Hs);
+  // destination rank and its (token, head) for the current row
+  int peer, td, hd;
+  if (p.to_heads) {
+    peer = h / p.heads_per_rank;
+    hd = h - peer * p.heads_per_rank;
+    td = p.rank * p.tokens_per_rank + t;
+  } else {
+    peer = t / p.tokens_per_rank;
+    td = t - peer * p.tokens_per_rank;
+    hd = p.rank * p.Hs + h;
   }
-  // the stores into a peer's memory are performed before this grid completes
-  __threadfence_system();
+  const char* src = static_cast<const char*>(p.src) + (long long)b * p.s_stride[0] * p.es + 16 * piece;
+  const long long dst_b = (long long)b * p.d_stride[0] * p.es + 16 * piece;
+  for (; row < r1;) {
+    uint4 v[U];
+    char* dst[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      dst[u] = nullptr;
+      if (row < r1) {
+        v[u] = __ldg(reinterpret_cast<const uint4*>(src + ((long long)t * p.s_stride[1] + (long long)h * p.s_stride[2]) * p.es));
+        dst[u] = static_cast<char*>(p.dst[peer]) + dst_b + ((long long)td * p.d_stride[1] + (long long)hd * p.d_stride[2]) * p.es;
+      }
+      // advance R rows: dt tokens and dh heads, carrying into the token
+      row += R;
+      t += dt;
+      h += dh;
+      const bool carry = h >= p.Hs;
+      if (carry) {
+        h -= p.Hs;
+        ++t;
+      }
+      if (p.to_heads) {
+        // the rank follows the head: hd counts heads within the rank's slice
+        td += dt + (carry ? 1 : 0);
+        hd += dh;
+        while (hd >= p.heads_per_rank) {
+          hd -= p.heads_per_rank;
+          ++peer;
+        }
+        if (carry) peer -= p.Hs / p.heads_per_rank;  // the head index wrapped past the last rank
+      } else {
+        // the rank follows the token: td counts tokens within the rank's shard
+        hd += dh;
+        if (carry) hd -= p.Hs;
+        td += dt + (carry ? 1 : 0);
+        while (td >= p.tokens_per_rank) {
+          td -= p.tokens_per_rank;
+          ++peer;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (dst[u]) *reinterpret_cast<uint4*>(dst[u]) = v[u];
+  }
 }
 
 }  // namespace
 
 int launch_exchange(const ExchangeDevParams& p, void* stream) {
-  const unsigned long long n = ((unsigned long long)p.Ls * (unsigned long long)p.Hs) << p.chunk_shift;
-  if (n == 0) return KREA_OK;
+  const long long rows = (long long)p.Ls * p.Hs;
+  if (rows == 0) return KREA_OK;
+  ExchangeDevParams q = p;
   // about 8 CTAs of 256 threads per SM (148 SMs) over the whole grid, split
-  // across the batch; each thread moves 4 pieces per loop iteration
-  const unsigned long long per_b = (n + 256ull * 4 - 1) / (256ull * 4);
-  const unsigned long long total = per_b * (unsigned long long)p.B;
-  const unsigned long long target = total < 1184ull ? total : 1184ull;
-  unsigned gx = (unsigned)((target + p.B - 1) / p.B);
-  if (gx == 0) gx = 1;
-  exchange_kernel<<<dim3(gx, (unsigned)p.B), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  // across the batch; each run a multiple of one step of rows
+  const int R = 256 >> p.chunk_shift;
+  long long gx = (1184 + p.B - 1) / p.B;
+  long long per = (rows + gx - 1) / gx;
+  per = (per + R - 1) / R * R;
+  gx = (rows + per - 1) / per;
+  q.rows_per_cta = per;
+  const dim3 grid((unsigned)gx, (unsigned)p.B);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (p.chunk_shift) {
+    case 3: exchange_kernel<3><<<grid, 256, 0, s>>>(q); break;
+    case 4: exchange_kernel<4><<<grid, 256, 0, s>>>(q); break;
+    case 5: exchange_kernel<5><<<grid, 256, 0, s>>>(q); break;
+    default: return KREA_ERR_UNSUPPORTED;
+  }
   return cudaGetLastError() == cudaSuccess ? KREA_OK : KREA_ERR_CUDA;
 }
 

@@ -81,6 +81,7 @@ struct ExchangeDevParams {
   int es;           // element bytes
   int to_heads;
   int rank, tokens_per_rank, heads_per_rank;
+  long long rows_per_cta;  // set by launch_exchange
 };
 int launch_exchange(const ExchangeDevParams& p, void* stream);
 int launch_rope_table(const int32_t* pos, int tokens, const int axes[3], double theta, float* table, void* stream);
