@@ -62,51 +62,66 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const int32_t* pos, int
   table[idx] = make_float2((float)c, (float)s);
 }
 
-// Grid (ceil(L / 128), H, B), 512 threads = 16 warps x 8 rows of the CTA's
-// 128-token block. A row of d channels is held by d/8 lanes, 8 channels (16
-// bytes) each, so one warp access covers 32 / (d/8) whole rows: 512 contiguous
-// bytes per row pair at d = 128. Channel pairs (2i, 2i+1) never straddle lanes.
+// 512 threads = 16 warps. A row (token, head) of d channels is held by d/8
+// lanes, 8 channels (16 bytes) each, so one warp access covers RPW = 32 / (d/8)
+// rows. Channel pairs (2i, 2i+1) never straddle lanes. Each thread makes STEPS =
+// 8 / RPW accesses, every load issued before the first use:
+//  - without codes, grid (ceil(L / (16 RPW)), ceil(H / STEPS), B): a thread keeps
+//    one token and steps through STEPS consecutive heads, so its rotary table
+//    entries are loaded once for all of them;
+//  - with codes, grid (ceil(L / 128), H, B): the CTA holds one head's whole
+//    128-token block (the scale is its absmax), a thread steps through tokens.
 template <bool BF16, int D, bool CODES>
 __global__ void __launch_bounds__(512, CODES ? 1 : 2) prologue_kernel(PrologueDevParams p) {
   constexpr int LPR = D / 8;       // lanes per row
   constexpr int RPW = 32 / LPR;    // rows per warp access
-  constexpr int STEPS = 8 / RPW;   // accesses per warp for its 8 rows
-  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  constexpr int STEPS = 8 / RPW;   // accesses per thread
+  const int b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane / LPR, li = lane % LPR;
   const int c0 = 8 * li;            // this lane's channels c0 .. c0 + 7
   const int pj0 = c0 / 2;           // and its rotary pairs pj0 .. pj0 + 3
+  // the (token, head) of step st
+  auto token_of = [&](int st) {
+    return CODES ? (int)blockIdx.x * kTile + warp * 8 + st * RPW + sub : (int)blockIdx.x * (16 * RPW) + warp * RPW + sub;
+  };
+  auto head_of = [&](int st) { return CODES ? (int)blockIdx.y : (int)blockIdx.y * STEPS + st; };
   __shared__ float red[16];
-  // where this head's rows go: y, or a peer's buffer of the sequence <-> head exchange
-  uint16_t* ybase = static_cast<uint16_t*>(p.y);
-  int hy = h;
-  if (p.heads_per_peer > 0) {
-    const int j = h / p.heads_per_peer;
-    ybase = static_cast<uint16_t*>(p.y_peer[j]);
-    hy = h - j * p.heads_per_peer;
-  }
   uint64_t g2[4];  // the weights as f32 pairs: the arithmetic below is packed (two lanes per op)
 #pragma unroll
   for (int j = 0; j < 4; ++j)
     g2[j] = p.gamma ? ptx::f2(p.gamma[c0 + 2 * j], p.gamma[c0 + 2 * j + 1]) : ptx::f2(1.0f, 1.0f);
   float keep[CODES ? STEPS : 1][8];  // stored values, for the codes
   float amax = 0.f;
-  uint4 raw[STEPS];  // every load of the thread is issued before the first use
+  uint4 raw[STEPS];
 #pragma unroll
   for (int st = 0; st < STEPS; ++st) {
-    const int t = blk * kTile + warp * 8 + st * RPW + sub;
-    raw[st] = t < p.L ? *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + b * p.x_stride[0] +
-                                                        (long long)t * p.x_stride[1] + h * p.x_stride[2] + c0)
-                      : make_uint4(0u, 0u, 0u, 0u);
+    const int t = token_of(st), hh = head_of(st);
+    raw[st] = t < p.L && hh < p.H
+                  ? *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + b * p.x_stride[0] +
+                                                    (long long)t * p.x_stride[1] + hh * p.x_stride[2] + c0)
+                  : make_uint4(0u, 0u, 0u, 0u);
+  }
+  // without codes every step has the same token: its table entries, once
+  float4 cs_tok[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+  if constexpr (!CODES) {
+    const int t = token_of(0);
+    if (t < p.L) {
+      const float4* tab =
+          reinterpret_cast<const float4*>(p.table + 2LL * (((long long)t + p.token_offset) * p.n_pairs + pj0));
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2)
+        if (pj0 + 2 * q2 < p.n_pairs) cs_tok[q2] = tab[q2];
+    }
   }
 #pragma unroll
   for (int st = 0; st < STEPS; ++st) {
-    const int t = blk * kTile + warp * 8 + st * RPW + sub;
-    const bool live = t < p.L;
+    const int t = token_of(st), hh = head_of(st);
+    const bool live = t < p.L && hh < p.H;
     uint64_t x2[4];  // channel pairs (2j, 2j+1) of this lane, as f32 pairs
     float ss = 0.f;
     {
-      const uint4 u = raw[st];  // zero for rows past L
+      const uint4 u = raw[st];  // zero for rows past L or H
       const uint16_t* e = reinterpret_cast<const uint16_t*>(&u);
       uint64_t acc = ptx::f2(0.f, 0.f);
 #pragma unroll
@@ -127,11 +142,11 @@ __global__ void __launch_bounds__(512, CODES ? 1 : 2) prologue_kernel(PrologueDe
 #pragma unroll
       for (int j = 0; j < 4; ++j) x2[j] = ptx::mul2(ptx::mul2(x2[j], r2), g2[j]);
       const long long tg = (long long)t + p.token_offset;  // token in the whole sequence
-      const float4* tab = reinterpret_cast<const float4*>(p.table + 2LL * (tg * p.n_pairs + pj0));
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {  // two pairs per 16-byte table load
+      for (int q2 = 0; q2 < 2; ++q2) {  // two pairs per 16-byte table entry
         if (pj0 + 2 * q2 >= p.n_pairs) break;
-        const float4 cs = tab[q2];
+        const float4 cs =
+            CODES ? reinterpret_cast<const float4*>(p.table + 2LL * (tg * p.n_pairs + pj0))[q2] : cs_tok[q2];
         // (a0, a1) -> (a0 c - a1 s, a0 s + a1 c) = (a0, a0) (c, s) + (a1, a1) (-s, c)
         float a0, a1, b0, b1;
         ptx::unf2(x2[2 * q2], a0, a1);
@@ -139,6 +154,14 @@ __global__ void __launch_bounds__(512, CODES ? 1 : 2) prologue_kernel(PrologueDe
         x2[2 * q2] = ptx::fma2(ptx::f2(a1, a1), ptx::f2(-cs.y, cs.x), ptx::mul2(ptx::f2(a0, a0), ptx::f2(cs.x, cs.y)));
         x2[2 * q2 + 1] =
             ptx::fma2(ptx::f2(b1, b1), ptx::f2(-cs.w, cs.z), ptx::mul2(ptx::f2(b0, b0), ptx::f2(cs.z, cs.w)));
+      }
+      // where this head's row goes: y, or a peer's buffer of the sequence <-> head exchange
+      uint16_t* ybase = static_cast<uint16_t*>(p.y);
+      int hy = hh;
+      if (p.heads_per_peer > 0) {
+        const int j = hh / p.heads_per_peer;
+        ybase = static_cast<uint16_t*>(p.y_peer[j]);
+        hy = hh - j * p.heads_per_peer;
       }
       float x[8];
 #pragma unroll
@@ -170,10 +193,11 @@ __global__ void __launch_bounds__(512, CODES ? 1 : 2) prologue_kernel(PrologueDe
   for (int w = 1; w < 16; ++w) amax = fmaxf(amax, red[w]);
   const float scale = __fdiv_rn(amax, 127.0f);
   const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
-  if (threadIdx.x == 0) p.scales[((long long)b * p.H + h) * p.nt + blk] = scale;
+  const int h = blockIdx.y;
+  if (threadIdx.x == 0) p.scales[((long long)b * p.H + h) * p.nt + blockIdx.x] = scale;
 #pragma unroll
   for (int st = 0; st < STEPS; ++st) {
-    const int t = blk * kTile + warp * 8 + st * RPW + sub;
+    const int t = token_of(st);
     if (t >= p.L) continue;
     uint2 u;
     int8_t* e = reinterpret_cast<int8_t*>(&u);
@@ -201,20 +225,23 @@ int launch_rope_table(const int32_t* pos, int tokens, const int axes[3], double 
 
 int launch_prologue(const PrologueDevParams& p, bool bf16, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const dim3 grid((unsigned)p.nt, (unsigned)p.H, (unsigned)p.B);
   const bool codes = p.codes != nullptr;
+  if (p.d != 128 && p.d != 64) return KREA_ERR_UNSUPPORTED;
+  // rows per warp access 256 / d, accesses per thread 8 / that (see the kernel)
+  const int rpw = 256 / p.d, steps = 8 / rpw;
+  const dim3 grid = codes ? dim3((unsigned)p.nt, (unsigned)p.H, (unsigned)p.B)
+                          : dim3((unsigned)((p.L + 16 * rpw - 1) / (16 * rpw)), (unsigned)((p.H + steps - 1) / steps),
+                                 (unsigned)p.B);
   if (p.d == 128) {
     if (bf16) codes ? prologue_kernel<true, 128, true><<<grid, 512, 0, s>>>(p)
                     : prologue_kernel<true, 128, false><<<grid, 512, 0, s>>>(p);
     else codes ? prologue_kernel<false, 128, true><<<grid, 512, 0, s>>>(p)
                : prologue_kernel<false, 128, false><<<grid, 512, 0, s>>>(p);
-  } else if (p.d == 64) {
+  } else {
     if (bf16) codes ? prologue_kernel<true, 64, true><<<grid, 512, 0, s>>>(p)
                     : prologue_kernel<true, 64, false><<<grid, 512, 0, s>>>(p);
     else codes ? prologue_kernel<false, 64, true><<<grid, 512, 0, s>>>(p)
                : prologue_kernel<false, 64, false><<<grid, 512, 0, s>>>(p);
-  } else {
-    return KREA_ERR_UNSUPPORTED;
   }
   return cudaGetLastError() == cudaSuccess ? KREA_OK : KREA_ERR_CUDA;
 }
