@@ -196,6 +196,13 @@ class PeerMapping:
 
 
 # ----------------------------------------------------------------------------- one rank's end
+def _core(q, k, v, gate, **kw):
+    """The attention core on this rank's heads over the whole sequence."""
+    from . import attention
+
+    return attention(q, k, v, gate, **kw)
+
+
 class SequenceParallelAttention:
     """The attention core for a block whose activations are split by token over
     the ranks of `group` (None: one rank). Per call: q and k through the QK
@@ -204,9 +211,13 @@ class SequenceParallelAttention:
     back to the token shards. Buffers are allocated once; the handles of other
     ranks' buffers are exchanged with all_gather_object when world > 1."""
 
+    # how buffers other ranks map are made and opened (CUDA IPC)
+    buffer_cls = PeerBuffer
+    mapping_cls = PeerMapping
+
     def __init__(self, batch: int, tokens_per_rank: int, q_heads: int, kv_heads: int, head_dim: int,
                  dtype: torch.dtype = torch.bfloat16, out_dtype: torch.dtype = torch.float32, group=None,
-                 with_gate: bool = True):
+                 with_gate: bool = True, device="cuda"):
         import torch.distributed as dist
 
         self.group = group
@@ -228,11 +239,11 @@ class SequenceParallelAttention:
         self.local, self.dests, self._keep = {}, {}, []
         if W == 1:
             for name, (shape, dt) in shapes.items():
-                self.local[name] = torch.empty(shape, dtype=dt, device="cuda")
+                self.local[name] = torch.empty(shape, dtype=dt, device=device)
                 self.dests[name] = Destinations.of([self.local[name]])
-            self.o_heads = torch.empty((batch, L, q_heads, head_dim), dtype=out_dtype, device="cuda")
+            self.o_heads = torch.empty((batch, L, q_heads, head_dim), dtype=out_dtype, device=device)
             return
-        own = {name: PeerBuffer(shape, dt) for name, (shape, dt) in shapes.items()}
+        own = {name: self.buffer_cls(shape, dt) for name, (shape, dt) in shapes.items()}
         self._keep.append(own)
         handles = {name: b.handle_bytes() for name, b in own.items()}
         gathered: List[dict] = [None] * W
@@ -243,14 +254,14 @@ class SequenceParallelAttention:
                 if j == self.rank:
                     ptrs.append(own[name].ptr)
                 else:
-                    m = PeerMapping(gathered[j][name])
+                    m = self.mapping_cls(gathered[j][name])
                     self._keep.append(m)
                     ptrs.append(m.ptr)
             self.local[name] = own[name].tensor()
             strides = torch.empty(shape, dtype=dt, device="meta").stride()
             self.dests[name] = Destinations(ptrs, strides, dt)
-        self.o_heads = torch.empty((batch, L, q_heads // W, head_dim), dtype=out_dtype, device="cuda")
-        self._flag = torch.zeros(1, dtype=torch.float32, device="cuda")
+        self.o_heads = torch.empty((batch, L, q_heads // W, head_dim), dtype=out_dtype, device=device)
+        self._flag = torch.zeros(1, dtype=torch.float32, device=device)
 
     def _barrier(self) -> None:
         """Stream-ordered: work after it on this stream starts once every rank's
@@ -267,8 +278,6 @@ class SequenceParallelAttention:
         """q, k raw (before RMSNorm and RoPE), v, gate: this rank's token shards
         [B, Ls, H, d]. Returns this rank's token shard of the output [B, Ls, Hq, d]
         (a buffer reused by the next call)."""
-        from . import attention
-
         if (gate is None) != ("gate" not in self.local):
             raise ValueError("gate given to an instance built without one, or missing")
         r = self.rank
@@ -279,8 +288,8 @@ class SequenceParallelAttention:
         if gate is not None:
             seq_to_heads(gate, self.dests["gate"], r)
         self._barrier()  # this rank's head shards are complete
-        attention(self.local["q"], self.local["k"], self.local["v"], self.local.get("gate"), text_len=text_len,
-                  grid_h=grid_h, grid_w=grid_w, mode=mode, out=self.o_heads, **opts)
+        _core(self.local["q"], self.local["k"], self.local["v"], self.local.get("gate"), text_len=text_len,
+              grid_h=grid_h, grid_w=grid_w, mode=mode, out=self.o_heads, **opts)
         heads_to_seq(self.o_heads, self.dests["out"], r)
         self._barrier()  # this rank's token shard of the output is complete
         return self.local["out"]

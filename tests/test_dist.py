@@ -148,3 +148,106 @@ def test_sequence_parallel_ranges():
 
     with pytest.raises(ValueError):
         seqpar.head_range(12, 5, 0)
+
+
+def _sequence_parallel_class_worker(rank, world, port, shared_dir, results):
+    """SequenceParallelAttention with world = 2 on gloo ranks. Its host logic runs
+    unchanged: buffer allocation, the exchange of handles, the tables of
+    destinations in rank order, the barriers. What runs on a GPU is replaced:
+    buffers are file-backed shared arrays (the handle is the path), the pushes
+    write into them by the layout rule of the C ABI, and the core and the
+    prologue are the fp64 oracle."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import dataclasses
+        import json
+        import tempfile
+
+        import numpy as np
+
+        from diffusion_transformer_attention_bidirectional_b200 import seqpar
+        from oracle import krea_oracle as ko
+        from synth import inputs as S
+
+        arrays = {}  # fake "device pointer" -> the shared array it addresses
+
+        class FileBuffer:
+            def __init__(self, shape, dtype):
+                fd, self.path = tempfile.mkstemp(dir=shared_dir)
+                os.close(fd)
+                self.shape = tuple(shape)
+                self.arr = np.memmap(self.path, dtype=np.float64, mode="w+", shape=self.shape)
+                self.arr[...] = np.nan
+                self.ptr = id(self.arr)
+                arrays[self.ptr] = self.arr
+
+            def handle_bytes(self):
+                return json.dumps([self.path, self.shape]).encode()
+
+            def tensor(self):
+                return torch.from_numpy(self.arr)
+
+        class FileMapping:
+            def __init__(self, handle):
+                path, shape = json.loads(handle.decode())
+                self.arr = np.memmap(path, dtype=np.float64, mode="r+", shape=tuple(shape))
+                self.ptr = id(self.arr)
+                arrays[self.ptr] = self.arr
+
+        case = S.Case("seqpar_cls", 1, 4, 2, 64, 16, 8, 8, dtype="f16", mode="scanline", window=3, gate=True,
+                      prologue=True, seed=9)
+        L, Ls = case.seq_len, case.seq_len // world
+        pos = ko.rope_positions(case.text_len, case.grid_h, case.grid_w)
+
+        def push_heads(y, dests, r):  # the rule of krea_attn_seq_to_heads
+            H = y.shape[2]
+            hpr = H // dests.world
+            for h in range(H):
+                arrays[dests.ptrs[h // hpr]][:, r * Ls:(r + 1) * Ls, h % hpr] = y[:, :, h]
+
+        def fake_prologue(x, table, dests, r, gamma=None, rope=None):
+            push_heads(ko.qk_prologue(x, table[r * Ls:(r + 1) * Ls]), dests, r)
+
+        def fake_seq_to_heads(x, dests, r):
+            push_heads(np.asarray(x, dtype=np.float64), dests, r)
+
+        def fake_heads_to_seq(y, dests, r):  # the rule of krea_attn_heads_to_seq
+            y = np.asarray(y)
+            Hr = y.shape[2]
+            for t in range(y.shape[1]):
+                arrays[dests.ptrs[t // Ls]][:, t % Ls, r * Hr:(r + 1) * Hr] = y[:, t]
+
+        def fake_core(q, k, v, gate, *, out, **kw):
+            sub = dataclasses.replace(case, q_heads=q.shape[2], kv_heads=k.shape[2])
+            out[...] = torch.from_numpy(ko.attention(sub, q, k, v, gate)["out"])
+
+        seqpar.qk_prologue_to_heads = fake_prologue
+        seqpar.seq_to_heads = fake_seq_to_heads
+        seqpar.heads_to_seq = fake_heads_to_seq
+        seqpar._core = fake_core
+        seqpar.SequenceParallelAttention.buffer_cls = FileBuffer
+        seqpar.SequenceParallelAttention.mapping_cls = FileMapping
+
+        spa = seqpar.SequenceParallelAttention(1, Ls, case.q_heads, case.kv_heads, case.head_dim,
+                                               dtype=torch.float64, out_dtype=torch.float64, device="cpu")
+        assert spa.world == world and spa.rank == rank
+        q, k, v, g = S.make_inputs(case)
+        t0, t1 = seqpar.token_range(Ls, rank)
+        out = spa(q[:, t0:t1], k[:, t0:t1], v[:, t0:t1].double(), g[:, t0:t1].double(), pos,
+                  text_len=case.text_len, grid_h=case.grid_h, grid_w=case.grid_w, mode="scanline", window=3)
+        full = ko.attention(case, ko.qk_prologue(q, pos), ko.qk_prologue(k, pos), v, g)["out"]
+        results[rank] = float(np.abs(out.numpy() - full[:, t0:t1]).max())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sequence_parallel_attention_two_ranks_host_logic(tmp_path):
+    world = 2
+    mgr = mp.Manager()
+    results = mgr.dict()
+    mp.spawn(_sequence_parallel_class_worker, args=(world, _free_port(), str(tmp_path), results), nprocs=world,
+             join=True)
+    for r in range(world):
+        assert results[r] < 1e-12, results[r]
