@@ -284,7 +284,7 @@ int krea_attn_map_size(int text_len, int grid_h, int grid_w, int mode, const kre
   int rc = make_geometry(text_len, grid_h, grid_w, mode, params, &g);
   if (rc != KREA_OK) return rc;
   HostMap hm;
-  rc = build_map(g, &hm);
+  rc = build_map(g, &hm, /*quiet=*/true);
   if (rc != KREA_OK) return rc;
   if (n_tiles) *n_tiles = hm.n_tiles;
   if (nnz) *nnz = (int32_t)hm.entries.size();

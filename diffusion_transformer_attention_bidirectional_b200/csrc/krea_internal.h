@@ -40,8 +40,10 @@ struct HostMap {
   int n_int8 = 0;
 };
 
-// Builds a map (tilemap.cpp). Returns KREA_OK or an error code.
-int build_map(const Geometry& g, HostMap* out);
+// Builds a map (tilemap.cpp). Returns KREA_OK or an error code. With the
+// environment variable KREA_ATTN_LOG set (not "0"), prints one line per map to
+// stderr unless `quiet` (a size query).
+int build_map(const Geometry& g, HostMap* out, bool quiet = false);
 
 // Builds the map on the device (mapgen.cu): row_ptr[n_tiles + 1], and either packed
 // entries ((key tile << 2) | kind, packed != nullptr) or col / kind arrays. Nothing

@@ -7,7 +7,9 @@
 // cache of "Krea 2 Scanline Attention", section "Where people get burned".
 #include <algorithm>
 #include <cmath>
+#include <cstdio>
 #include <cstdlib>
+#include <cstring>
 
 #include "krea_internal.h"
 
@@ -166,7 +168,40 @@ int make_geometry(int text_len, int grid_h, int grid_w, int mode, const krea_att
   return KREA_OK;
 }
 
-int build_map(const Geometry& g, HostMap* out) {
+namespace {
+
+// KREA_ATTN_LOG set to anything but "0": one line on stderr per map built, the
+// counterpart of the pages' console lines that confirm the path is active.
+bool log_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("KREA_ATTN_LOG");
+    return e != nullptr && *e != '\0' && std::strcmp(e, "0") != 0;
+  }();
+  return on;
+}
+
+void log_map(const Geometry& g, const HostMap& m) {
+  long masked = 0;
+  for (int32_t e : m.entries) masked += (e & KREA_KIND_MASKED) ? 1 : 0;
+  const long pairs = (long)m.n_tiles * m.n_tiles;
+  const long active = (long)m.entries.size();
+  char extra[96] = "";
+  if (g.mode == KREA_MODE_SCANLINE)
+    std::snprintf(extra, sizeof(extra), " text_pad=%d window=%d tile_aligned=%d", g.Pt, g.window, g.tile_aligned);
+  else if (g.mode == KREA_MODE_TILEMIX)
+    std::snprintf(extra, sizeof(extra), " pattern=%s percentage=%g band=%d",
+                  g.pattern == KREA_PATTERN_ZERO ? "zero" : g.pattern == KREA_PATTERN_ONE ? "one" : "band",
+                  (double)g.percentage, g.band_blocks);
+  const char* name = g.mode == KREA_MODE_SCANLINE ? "scanline" : g.mode == KREA_MODE_TILEMIX ? "tilemix" : "dense";
+  std::fprintf(stderr,
+               "[krea_attn] map %s T=%d grid=%dx%d%s: %dx%d tiles, %ld active (%.1f%%), %d int8, %ld masked\n",
+               name, g.T, g.H, g.W, extra, m.n_tiles, m.n_tiles, active,
+               pairs > 0 ? 100.0 * (double)active / (double)pairs : 0.0, m.n_int8, masked);
+}
+
+}  // namespace
+
+int build_map(const Geometry& g, HostMap* out, bool quiet) {
   if (!out) return KREA_ERR_INVALID_ARG;
   out->row_ptr.clear();
   out->entries.clear();
@@ -178,6 +213,7 @@ int build_map(const Geometry& g, HostMap* out) {
     case KREA_MODE_TILEMIX: build_tilemix(g, out); break;
     default: build_dense(g, out); break;
   }
+  if (!quiet && log_enabled()) log_map(g, *out);
   return KREA_OK;
 }
 

@@ -198,3 +198,28 @@ def test_exchange_arguments_rejected_without_gpu():
     assert L.krea_attn_ipc_open(h, ctypes.byref(p)) == _lib.ERR_NO_DEVICE
     assert L.krea_attn_ipc_free(None) == _lib.ERR_INVALID_ARG
     assert L.krea_attn_ipc_close(None) == _lib.ERR_INVALID_ARG
+
+
+def test_map_log_lines():
+    # KREA_ATTN_LOG prints one line per map built (not for size queries) with the
+    # map's tile counts; unset or "0", nothing
+    import sys
+
+    prog = ("import diffusion_transformer_attention_bidirectional_b200 as K\n"
+            "K.get_map('scanline', 512, 64, 64, window=11)\n"
+            "K.get_map('tilemix', 512, 128, 128, pattern='band', percentage=0.5)\n")
+
+    def run(value):
+        env = dict(os.environ)
+        env.pop("KREA_ATTN_LOG", None)
+        if value is not None:
+            env["KREA_ATTN_LOG"] = value
+        r = subprocess.run([sys.executable, "-c", prog], cwd=ROOT, env=env, capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+        return [ln for ln in r.stderr.splitlines() if ln.startswith("[krea_attn]")]
+
+    lines = run("1")
+    assert len(lines) == 2
+    assert "map scanline T=512 grid=64x64" in lines[0] and "36x36 tiles, 484 active" in lines[0]
+    assert "map tilemix" in lines[1] and "17424 active" in lines[1] and "7938 int8" in lines[1]
+    assert run("0") == [] and run(None) == []
