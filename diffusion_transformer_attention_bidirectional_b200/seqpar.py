@@ -209,7 +209,9 @@ class SequenceParallelAttention:
     prologue straight into the owners' head shards, v and gate copied the same
     way, the core on this rank's heads over the whole sequence, its output pushed
     back to the token shards. Buffers are allocated once; the handles of other
-    ranks' buffers are exchanged with all_gather_object when world > 1."""
+    ranks' buffers are exchanged with all_gather_object when world > 1, so each
+    process sets its own device (torch.cuda.set_device) before building one, and
+    all ranks build theirs together. Ranks of one node only (CUDA IPC)."""
 
     # how buffers other ranks map are made and opened (CUDA IPC)
     buffer_cls = PeerBuffer
