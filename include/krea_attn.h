@@ -233,7 +233,17 @@ KREA_API int krea_attn_qk_prologue(const void* x, void* y, const float* gamma, c
  * orders the ranks around it: no rank may read a destination before every rank's
  * exchange into it has completed (a stream-ordered barrier, e.g. a one-element
  * all-reduce), and no rank may overwrite a destination that its owner still
- * reads. */
+ * reads. The stores are performed when the launch completes on `stream`.
+ *
+ * Ownership: the caller owns the source, every destination and the stream; the
+ * library keeps no pointer after the call returns. Source and destinations must
+ * not overlap. Errors, returned before anything is launched or written:
+ * KREA_ERR_INVALID_ARG (world, rank, tokens_per_rank or reserved out of range,
+ * a NULL or misaligned pointer, a stride that is not a positive multiple of 16
+ * bytes, heads not divisible by world, an unknown dtype), KREA_ERR_UNSUPPORTED
+ * (head_dim not 64 or 128; fp32 into the prologue), KREA_ERR_TOO_LARGE,
+ * KREA_ERR_NO_DEVICE; KREA_ERR_CUDA if the launch fails. Destination sizes are
+ * not checked: each dst[j] must hold the shape the rule below writes. */
 #define KREA_EXCHANGE_MAX_RANKS 16
 typedef struct {
   int32_t world;            /* ranks sharing the sequence, 1 .. KREA_EXCHANGE_MAX_RANKS */
@@ -279,7 +289,9 @@ KREA_API int krea_attn_qk_prologue_to_heads(const void* x, const float* gamma, c
  * handle (KREA_IPC_HANDLE_BYTES opaque bytes) to `handle`; krea_attn_ipc_free
  * releases it. krea_attn_ipc_open maps another process's handle into this one
  * (not one of this process's own allocations) and krea_attn_ipc_close unmaps
- * it. Failures return KREA_ERR_CUDA with nothing allocated or mapped. */
+ * it. NULL arguments or zero bytes return KREA_ERR_INVALID_ARG, a missing sm_100
+ * device KREA_ERR_NO_DEVICE; CUDA failures return KREA_ERR_CUDA with nothing
+ * allocated or mapped. */
 #define KREA_IPC_HANDLE_BYTES 64
 KREA_API int krea_attn_ipc_alloc(size_t bytes, void** ptr, void* handle);
 KREA_API int krea_attn_ipc_free(void* ptr);
