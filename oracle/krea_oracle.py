@@ -52,8 +52,11 @@ at (0, r, c). Parity of this step is pinned by the closed forms and the
 rotation identities in the tests.
 
 Parity note: the INT8 quantisation scheme is fixed by the specification, not by
-the pages, so the INT8 path is pinned only by its error bound and by the pages'
-invariants (pattern zero equals dense, smooth_k leaves FP16 results unchanged).
+the pages. The INT8 branch of `attention` is pinned by a per-row, per-tile
+brute force of that scheme (centring, block scales, round-half-even codes, the
+dequantised INT8 scores mixed with FP16 scores in one softmax), the key mean by
+a closed form, and both by the pages' invariants (pattern zero equals dense,
+smooth_k leaves FP16 results unchanged) and the per-pair INT8 error bound.
 """
 from __future__ import annotations
 

@@ -63,6 +63,8 @@ def compare(case, out_gpu, q, k, v, g, rows=None, heads=None, tol=None):
     assert np.all(np.isfinite(got))
     err = np.max(np.abs(got - ref))
     scale = max(1.0, float(np.max(np.abs(ref))))
+    print(f"[parity] {case.name} {case.mode} {case.dtype} T={case.text_len} {case.grid_h}x{case.grid_w}: "
+          f"max |gpu - oracle| = {err:.3e} (tol {tol * scale:.3e})")
     assert err <= tol * scale, f"max abs err {err:.3e} > {tol * scale:.3e}"
     return err
 

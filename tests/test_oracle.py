@@ -476,3 +476,122 @@ def test_backward_closed_forms():
     # a row's weights do not change when every key moves by the same vector (each
     # score of the row shifts by one constant): sum_j dS_ij = 0, so sum_j dK_j = 0
     assert np.allclose(gr["dk"].sum(axis=1), 0.0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- INT8 tiles and the key mean
+
+def _brute_int8_attention(q, k, v, T, band_blocks, int8_tile, smooth_k, scale):
+    """TileMix attention written out per query row and key tile, straight from the
+    definitions ("Krea 2 TileMix Attention (FP16/INT8 tiles)", sections "What it
+    actually patches" and "The inputs that matter", with the symmetric
+    per-(batch, head, 128-token block) absmax/127 scheme the specification fixes):
+
+      mu[b, g, c] = (1 / L) sum_t k[b, t, g, c]        (smooth_k; 0 otherwise)
+      kc = k - mu                                      (used by FP16 and INT8 tiles)
+      S(block) = max |x| over the block's tokens and channels / 127
+      X8 = round_half_even(x / S) clamped to [-127, 127]   (0 when S = 0)
+      s(t, j) = S_q(t) S_k(j) sum_c Q8[t, c] K8[j, c]   on an INT8 tile
+              = sum_c q[t, c] kc[j, c]                 on an FP16 tile
+      out[t] = sum_j softmax_j(scale s(t, j)) v[j]      (every key admitted)
+
+    Each piece is computed here on its own, with loops over tokens, blocks and
+    tiles; int8_tile(a, b) says whether tile (query tile a, key tile b) is INT8."""
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    rep = Hq // Hkv
+    mu = np.zeros((B, Hkv, d))
+    if smooth_k:
+        for b in range(B):
+            for g in range(Hkv):
+                acc = np.zeros(d)
+                for t in range(L):
+                    acc += k[b, t, g]
+                mu[b, g] = acc / L
+    kc = k - mu[:, None]
+
+    def codes_and_scales(x):
+        _, _, H, _ = x.shape
+        nb = (L + 127) // 128
+        c8 = np.zeros(x.shape)
+        sc = np.zeros((B, H, nb))
+        for b in range(B):
+            for h in range(H):
+                for j in range(nb):
+                    blk = x[b, 128 * j:128 * j + 128, h]
+                    amax = max(abs(float(e)) for e in blk.ravel())
+                    s = amax / 127.0
+                    sc[b, h, j] = s
+                    if s > 0:
+                        for r in range(blk.shape[0]):
+                            for c in range(d):
+                                c8[b, 128 * j + r, h, c] = min(127, max(-127, round(float(blk[r, c]) / s)))
+        return c8, sc
+
+    q8, sq = codes_and_scales(q)
+    k8, sk = codes_and_scales(kc)
+    out = np.zeros_like(q)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // rep
+            for t in range(L):
+                a = t // 128
+                s = np.empty(L)
+                for kb in range(0, L, 128):
+                    j = np.arange(kb, min(L, kb + 128))
+                    if int8_tile(a, kb // 128):
+                        s[j] = sq[b, h, a] * sk[b, g, kb // 128] * (k8[b, j, g] @ q8[b, t, h])
+                    else:
+                        s[j] = kc[b, j, g] @ q[b, t, h]
+                s = scale * s
+                w = np.exp(s - s.max())
+                out[b, t, h] = (w / w.sum()) @ v[b, :, g]
+    return out
+
+
+@pytest.mark.parametrize("pattern,smooth_k", [("one", True), ("one", False), ("band", True)])
+def test_int8_tiles_brute_force(pattern, smooth_k):
+    # 20 text tokens + 24 x 24 image tokens = 596 tokens: 5 tiles, the last one a
+    # ragged tail (84 tokens) that is both INT8 and masked in the exported map.
+    # K carries a per-channel offset, so the centring moves the INT8 codes.
+    c = Case("i8", 1, 2, 1, 16, 20, 24, 24, dtype="f16", mode="tilemix", seed=41, qk_dist="normal_koffset",
+             pattern=pattern, percentage=0.5, band_blocks=0, smooth_k=smooth_k)
+    q, k, v, _ = make_inputs(c)
+    qd, kd, vd = f64(q), f64(k), f64(v)
+    kind = ko.tile_map(c).kind
+    assert kind[1, 4] == ko.KIND_INT8 | ko.KIND_MASKED  # the ragged tail tile is both
+    if pattern == "one":
+        # written from the page: text tiles and the band (here the diagonal) stay FP16,
+        # every other image-image tile goes to INT8
+        def int8_tile(a, b):
+            return a != 0 and b != 0 and a != b
+    else:
+        def int8_tile(a, b):
+            return bool(kind[a, b] & ko.KIND_INT8)
+    n8 = sum(int8_tile(a, b) for a in range(5) for b in range(5))
+    assert n8 == (12 if pattern == "one" else 8)
+    want = _brute_int8_attention(qd, kd, vd, c.text_len, c.band_blocks, int8_tile, smooth_k, 1 / math.sqrt(16))
+    got = ko.attention(c, q, k, v)["out"]
+    assert np.max(np.abs(got - want)) <= 1e-12
+    # and the INT8 tiles really change the result: with every tile FP16 the rows
+    # whose tiles hold INT8 scores differ by the quantisation error
+    zero = ko.attention(Case(**{**c.__dict__, "pattern": "zero"}), q, k, v)["out"]
+    assert np.max(np.abs(zero[:, 128:] - want[:, 128:])) > 1e-4
+    assert np.max(np.abs(zero[:, :128] - want[:, :128])) <= 1e-12  # text query tile: all FP16
+
+
+def test_key_mean_closed_form():
+    # keys c + (-1)^t x over an even number of tokens: the +x and -x rows cancel, so
+    # the mean over tokens is exactly c and the centred keys are (-1)^t x
+    rng = np.random.default_rng(3)
+    B, L, Hkv, d = 2, 10, 3, 8
+    cvec = rng.standard_normal((B, Hkv, d))
+    x = rng.standard_normal((B, 1, Hkv, d))
+    sign = np.array([(-1.0) ** t for t in range(L)])[None, :, None, None]
+    k = cvec[:, None] + sign * x
+    assert np.max(np.abs(ko.key_mean(k) - cvec)) <= 1e-15
+    kc, mu = ko.centred_keys(k, "f64")
+    assert np.max(np.abs(mu - cvec)) <= 1e-15
+    assert np.max(np.abs(kc - sign * x)) <= 1e-15
+    # a constant key sequence has itself as mean and centres to zero
+    kconst = np.broadcast_to(cvec[:, None], (B, 7, Hkv, d))
+    assert np.max(np.abs(ko.centred_keys(kconst, "f64")[0])) <= 1e-15
