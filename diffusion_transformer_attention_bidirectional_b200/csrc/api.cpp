@@ -228,6 +228,172 @@ WsLayout workspace_layout(int B, int L, int Hq, int Hkv, int d, int in_bytes, in
   return w;
 }
 
+static int run_quantize(const void* q, const void* k, const Geometry& g, const krea_attn_params_t* p,
+                        bool quant_q, void* workspace, size_t workspace_bytes, void* stream) {
+  const int es = elem_bytes(p->in_dtype);
+  WsLayout w = workspace_layout(p->batch, g.L, p->num_q_heads, p->num_kv_heads, p->head_dim, es,
+                                p->smooth_k);
+  if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return KREA_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  QuantDevParams qp;
+  std::memset(&qp, 0, sizeof(qp));
+  qp.q = q;
+  qp.k = k;
+  for (int i = 0; i < 3; ++i) {
+    qp.q_stride[i] = p->q_stride[i];
+    qp.k_stride[i] = p->k_stride[i];
+  }
+  qp.kc = p->smooth_k ? ws + w.kc : nullptr;
+  qp.q8 = reinterpret_cast<int8_t*>(ws + w.q8);
+  qp.k8 = reinterpret_cast<int8_t*>(ws + w.k8);
+  qp.sq = reinterpret_cast<float*>(ws + w.sq);
+  qp.sk = reinterpret_cast<float*>(ws + w.sk);
+  qp.mu = reinterpret_cast<float*>(ws + w.mu);
+  qp.part = reinterpret_cast<double*>(ws + w.part);
+  qp.B = p->batch;
+  qp.L = g.L;
+  qp.Hq = p->num_q_heads;
+  qp.Hkv = p->num_kv_heads;
+  qp.d = p->head_dim;
+  qp.nt = (g.L + kTile - 1) / kTile;
+  qp.n_chunks = w.n_chunks;
+  qp.chunk_tokens = w.chunk_tokens;
+  qp.smooth_k = p->smooth_k ? 1 : 0;
+  qp.quant_q = quant_q ? 1 : 0;
+  return launch_quantize(qp, p->in_dtype == KREA_BF16, stream);
+}
+
+int check_params(const krea_attn_params_t* p) { return check_common(p); }
+
+int check_device_sm100() { return check_device(); }
+
+int check_forward(const void* q, const void* k, const void* v, const void* gate, const void* out,
+                  const Geometry& g, const krea_attn_params_t* p, int* q_len) {
+  const int es = elem_bytes(p->in_dtype), oes = elem_bytes(p->out_dtype);
+  if (!q || !k || !v || !out) return KREA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (gate && !aligned16(gate)))
+    return KREA_ERR_INVALID_ARG;
+  if (!stride_ok(p->q_stride, es) || !stride_ok(p->k_stride, es) || !stride_ok(p->v_stride, es) ||
+      !stride_ok(p->out_stride, oes) || (gate && !stride_ok(p->gate_stride, es)))
+    return KREA_ERR_INVALID_ARG;
+  // query slice
+  if (p->q_start < 0 || p->q_start % kTile != 0 || p->q_start >= g.L || p->q_len < 0)
+    return KREA_ERR_INVALID_ARG;
+  const int n = p->q_len == 0 ? g.L - p->q_start : p->q_len;
+  if ((long)p->q_start + n > g.L) return KREA_ERR_INVALID_ARG;
+  if (p->lse && (reinterpret_cast<uintptr_t>(p->lse) & 3)) return KREA_ERR_INVALID_ARG;
+  *q_len = n;
+  return KREA_OK;
+}
+
+int launch_forward(const void* q, const void* k, const void* v, const void* gate, void* out, const Geometry& g,
+                   const krea_attn_params_t* p, int q_len, const int32_t* row_ptr, const int32_t* entries,
+                   bool use_int8, void* workspace, size_t workspace_bytes, void* stream) {
+  const int mode = g.mode;
+  const int es = elem_bytes(p->in_dtype), oes = elem_bytes(p->out_dtype);
+  const bool bf16 = p->in_dtype == KREA_BF16;
+  const CUtensorMapDataType tdt = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const int d = p->head_dim, B = p->batch, Hq = p->num_q_heads, Hkv = p->num_kv_heads;
+  use_int8 = use_int8 && mode == KREA_MODE_TILEMIX;
+  const bool centred = mode == KREA_MODE_TILEMIX && p->smooth_k;
+  if (use_int8 && d != 128) return KREA_ERR_UNSUPPORTED;
+
+  const void* k_src = k;
+  int64_t kc_stride[3];
+  for (int i = 0; i < 3; ++i) kc_stride[i] = p->k_stride[i];
+  const float* sq = nullptr;
+  const float* sk = nullptr;
+  AttnMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  int rc = KREA_OK;
+  if (use_int8 || centred) {
+    rc = run_quantize(q, k, g, p, use_int8, workspace, workspace_bytes, stream);
+    if (rc != KREA_OK) return rc;
+    WsLayout w = workspace_layout(B, g.L, Hq, Hkv, d, es, p->smooth_k);
+    char* ws = static_cast<char*>(workspace);
+    if (centred) {
+      k_src = ws + w.kc;
+      const int64_t cs[3] = {(int64_t)g.L * Hkv * d, (int64_t)Hkv * d, d};
+      for (int i = 0; i < 3; ++i) kc_stride[i] = cs[i];
+    }
+    if (use_int8) {
+      const int64_t s8q[3] = {(int64_t)g.L * Hq * d, (int64_t)Hq * d, d};
+      const int64_t s8k[3] = {(int64_t)g.L * Hkv * d, (int64_t)Hkv * d, d};
+      rc = make_tmap(&maps.q8, ws + w.q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Hq, g.L, B, s8q, 128);
+      if (rc == KREA_OK)
+        rc = make_tmap(&maps.k8, ws + w.k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Hkv, g.L, B, s8k, 128);
+      if (rc != KREA_OK) return rc;
+      sq = reinterpret_cast<const float*>(ws + w.sq);
+      sk = reinterpret_cast<const float*>(ws + w.sk);
+    }
+  }
+  const int box = 64;  // 64 x 16-bit = one 128-byte swizzle row
+  rc = make_tmap(&maps.q, q, tdt, es, d, Hq, g.L, B, p->q_stride, box);
+  if (rc == KREA_OK) rc = make_tmap(&maps.k, k_src, tdt, es, d, Hkv, g.L, B, kc_stride, box);
+  if (rc == KREA_OK) rc = make_tmap(&maps.v, v, tdt, es, d, Hkv, g.L, B, p->v_stride, box);
+  if (rc != KREA_OK) return rc;
+  // epilogue maps: gate (16-bit, 64 per 128-byte row) and out (fp32: 32, 16-bit: 64)
+  bool tma_out = make_tmap(&maps.out, out,
+                           p->out_dtype == KREA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : tdt, oes, d, Hq, g.L, B,
+                           p->out_stride, p->out_dtype == KREA_F32 ? 32 : 64) == KREA_OK;
+  if (tma_out && gate) tma_out = make_tmap(&maps.gate, gate, tdt, es, d, Hq, g.L, B, p->gate_stride, box) == KREA_OK;
+
+  AttnDevParams ap;
+  std::memset(&ap, 0, sizeof(ap));
+  ap.row_ptr = row_ptr;
+  ap.entries = entries;
+  ap.gate = gate;
+  ap.out = out;
+  ap.sq = sq;
+  ap.sk = sk;
+  ap.status = p->status;
+  for (int i = 0; i < 3; ++i) {
+    ap.gate_stride[i] = p->gate_stride[i];
+    ap.out_stride[i] = p->out_stride[i];
+  }
+  ap.B = B;
+  ap.Hq = Hq;
+  ap.Hkv = Hkv;
+  ap.d = d;
+  ap.rep = Hq / Hkv;
+  ap.nh = (ap.rep % 2 == 0) ? 2 : 1;
+  ap.npairs = ap.rep / ap.nh;
+  ap.T = g.T;
+  ap.N = g.N;
+  ap.Pt = g.Pt;
+  ap.L = g.L;
+  ap.W = g.W;
+  ap.H = g.H;
+  ap.window_half = g.window / 2;
+  ap.tile_aligned = (mode != KREA_MODE_SCANLINE) || g.tile_aligned;
+  ap.n_tiles = g.n_tiles;
+  ap.q_lo = p->q_start;
+  ap.q_hi = p->q_start + q_len;
+  // logical tiles holding the slice's first and last physical rows
+  auto slot_of = [&](int t) { return t < g.T ? t : t - g.T + g.Pt; };
+  const int t_first = slot_of(ap.q_lo) / kTile, t_last = slot_of(ap.q_hi - 1) / kTile;
+  ap.tile_begin = t_first;
+  ap.n_slice_tiles = t_last - t_first + 1;
+  // Scanline: text query rows see every key tile, image rows only the text and their
+  // window, so the text tiles' CTAs go first and no long row starts in the last wave.
+  {
+    const int text_tiles = (g.T + kTile - 1) / kTile;
+    ap.n_heavy = mode == KREA_MODE_SCANLINE
+                     ? std::max(0, std::min(ap.tile_begin + ap.n_slice_tiles, text_tiles) - ap.tile_begin)
+                     : 0;
+  }
+  ap.nt_scale = (g.L + kTile - 1) / kTile;
+  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt((float)d);
+  ap.scale_log2 = scale * 1.4426950408889634f;
+  ap.has_gate = gate != nullptr;
+  ap.out_f32 = p->out_dtype == KREA_F32;
+  ap.tma_out = tma_out ? 1 : 0;
+  ap.wait_limit = p->debug_wait_limit > 0 ? p->debug_wait_limit : (long long)2000000000LL;
+  ap.debug_flags = p->debug_flags;
+  ap.lse = p->lse;
+  return launch_attention(ap, maps, bf16, stream);
+}
+
 }  // namespace krea
 
 extern "C" {
@@ -579,41 +745,6 @@ int krea_attn_workspace_layout(int text_len, int grid_h, int grid_w, int mode,
   return KREA_OK;
 }
 
-static int run_quantize(const void* q, const void* k, const Geometry& g, const krea_attn_params_t* p,
-                        bool quant_q, void* stream) {
-  const int es = elem_bytes(p->in_dtype);
-  WsLayout w = workspace_layout(p->batch, g.L, p->num_q_heads, p->num_kv_heads, p->head_dim, es,
-                                p->smooth_k);
-  if (!p->workspace || p->workspace_bytes < w.total || !aligned16(p->workspace)) return KREA_ERR_WORKSPACE;
-  char* ws = static_cast<char*>(p->workspace);
-  QuantDevParams qp;
-  std::memset(&qp, 0, sizeof(qp));
-  qp.q = q;
-  qp.k = k;
-  for (int i = 0; i < 3; ++i) {
-    qp.q_stride[i] = p->q_stride[i];
-    qp.k_stride[i] = p->k_stride[i];
-  }
-  qp.kc = p->smooth_k ? ws + w.kc : nullptr;
-  qp.q8 = reinterpret_cast<int8_t*>(ws + w.q8);
-  qp.k8 = reinterpret_cast<int8_t*>(ws + w.k8);
-  qp.sq = reinterpret_cast<float*>(ws + w.sq);
-  qp.sk = reinterpret_cast<float*>(ws + w.sk);
-  qp.mu = reinterpret_cast<float*>(ws + w.mu);
-  qp.part = reinterpret_cast<double*>(ws + w.part);
-  qp.B = p->batch;
-  qp.L = g.L;
-  qp.Hq = p->num_q_heads;
-  qp.Hkv = p->num_kv_heads;
-  qp.d = p->head_dim;
-  qp.nt = (g.L + kTile - 1) / kTile;
-  qp.n_chunks = w.n_chunks;
-  qp.chunk_tokens = w.chunk_tokens;
-  qp.smooth_k = p->smooth_k ? 1 : 0;
-  qp.quant_q = quant_q ? 1 : 0;
-  return launch_quantize(qp, p->in_dtype == KREA_BF16, stream);
-}
-
 int krea_attn_quantize(const void* q, const void* k, int text_len, int grid_h, int grid_w,
                        const krea_attn_params_t* p, void* stream) {
   int rc = check_common(p);
@@ -626,7 +757,7 @@ int krea_attn_quantize(const void* q, const void* k, int text_len, int grid_h, i
   if (!stride_ok(p->q_stride, 2) || !stride_ok(p->k_stride, 2)) return KREA_ERR_INVALID_ARG;
   rc = check_device();
   if (rc != KREA_OK) return rc;
-  return run_quantize(q, k, g, p, true, stream);
+  return run_quantize(q, k, g, p, true, p->workspace, p->workspace_bytes, stream);
 }
 
 int krea_attn_fwd(const void* q, const void* k, const void* v, const void* gate, void* out,
@@ -637,127 +768,16 @@ int krea_attn_fwd(const void* q, const void* k, const void* v, const void* gate,
   Geometry g;
   rc = make_geometry(text_len, grid_h, grid_w, mode, p, &g);
   if (rc != KREA_OK) return rc;
-  const int es = elem_bytes(p->in_dtype), oes = elem_bytes(p->out_dtype);
-  if (!q || !k || !v || !out) return KREA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (gate && !aligned16(gate)))
-    return KREA_ERR_INVALID_ARG;
-  if (!stride_ok(p->q_stride, es) || !stride_ok(p->k_stride, es) || !stride_ok(p->v_stride, es) ||
-      !stride_ok(p->out_stride, oes) || (gate && !stride_ok(p->gate_stride, es)))
-    return KREA_ERR_INVALID_ARG;
-  // query slice
-  if (p->q_start < 0 || p->q_start % kTile != 0 || p->q_start >= g.L || p->q_len < 0)
-    return KREA_ERR_INVALID_ARG;
-  const int q_len = p->q_len == 0 ? g.L - p->q_start : p->q_len;
-  if ((long)p->q_start + q_len > g.L) return KREA_ERR_INVALID_ARG;
+  int q_len = 0;
+  rc = check_forward(q, k, v, gate, out, g, p, &q_len);
+  if (rc != KREA_OK) return rc;
   rc = check_device();
   if (rc != KREA_OK) return rc;
-
   MapEntry map;
   rc = get_device_map(g, &map);
   if (rc != KREA_OK) return rc;
-
-  const bool bf16 = p->in_dtype == KREA_BF16;
-  const CUtensorMapDataType tdt = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  const int d = p->head_dim, B = p->batch, Hq = p->num_q_heads, Hkv = p->num_kv_heads;
-  const bool use_int8 = mode == KREA_MODE_TILEMIX && map.n_int8 > 0;
-  const bool centred = mode == KREA_MODE_TILEMIX && p->smooth_k;
-  if (use_int8 && d != 128) return KREA_ERR_UNSUPPORTED;
-
-  const void* k_src = k;
-  int64_t kc_stride[3];
-  for (int i = 0; i < 3; ++i) kc_stride[i] = p->k_stride[i];
-  const float* sq = nullptr;
-  const float* sk = nullptr;
-  AttnMaps maps;
-  std::memset(&maps, 0, sizeof(maps));
-  CUtensorMap &tm_q = maps.q, &tm_k = maps.k, &tm_v = maps.v, &tm_q8 = maps.q8, &tm_k8 = maps.k8;
-  if (use_int8 || centred) {
-    rc = run_quantize(q, k, g, p, use_int8, stream);
-    if (rc != KREA_OK) return rc;
-    WsLayout w = workspace_layout(B, g.L, Hq, Hkv, d, es, p->smooth_k);
-    char* ws = static_cast<char*>(p->workspace);
-    if (centred) {
-      k_src = ws + w.kc;
-      const int64_t cs[3] = {(int64_t)g.L * Hkv * d, (int64_t)Hkv * d, d};
-      for (int i = 0; i < 3; ++i) kc_stride[i] = cs[i];
-    }
-    if (use_int8) {
-      const int64_t s8q[3] = {(int64_t)g.L * Hq * d, (int64_t)Hq * d, d};
-      const int64_t s8k[3] = {(int64_t)g.L * Hkv * d, (int64_t)Hkv * d, d};
-      rc = make_tmap(&tm_q8, ws + w.q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Hq, g.L, B, s8q, 128);
-      if (rc == KREA_OK)
-        rc = make_tmap(&tm_k8, ws + w.k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, Hkv, g.L, B, s8k, 128);
-      if (rc != KREA_OK) return rc;
-      sq = reinterpret_cast<const float*>(ws + w.sq);
-      sk = reinterpret_cast<const float*>(ws + w.sk);
-    }
-  }
-  const int box = 64;  // 64 x 16-bit = one 128-byte swizzle row
-  rc = make_tmap(&tm_q, q, tdt, es, d, Hq, g.L, B, p->q_stride, box);
-  if (rc == KREA_OK) rc = make_tmap(&tm_k, k_src, tdt, es, d, Hkv, g.L, B, kc_stride, box);
-  if (rc == KREA_OK) rc = make_tmap(&tm_v, v, tdt, es, d, Hkv, g.L, B, p->v_stride, box);
-  if (rc != KREA_OK) return rc;
-  // epilogue maps: gate (16-bit, 64 per 128-byte row) and out (fp32: 32, 16-bit: 64)
-  bool tma_out = make_tmap(&maps.out, out,
-                           p->out_dtype == KREA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : tdt, oes, d, Hq, g.L, B,
-                           p->out_stride, p->out_dtype == KREA_F32 ? 32 : 64) == KREA_OK;
-  if (tma_out && gate) tma_out = make_tmap(&maps.gate, gate, tdt, es, d, Hq, g.L, B, p->gate_stride, box) == KREA_OK;
-
-  AttnDevParams ap;
-  std::memset(&ap, 0, sizeof(ap));
-  ap.row_ptr = map.d_row_ptr;
-  ap.entries = map.d_entries;
-  ap.gate = gate;
-  ap.out = out;
-  ap.sq = sq;
-  ap.sk = sk;
-  ap.status = p->status;
-  for (int i = 0; i < 3; ++i) {
-    ap.gate_stride[i] = p->gate_stride[i];
-    ap.out_stride[i] = p->out_stride[i];
-  }
-  ap.B = B;
-  ap.Hq = Hq;
-  ap.Hkv = Hkv;
-  ap.d = d;
-  ap.rep = Hq / Hkv;
-  ap.nh = (ap.rep % 2 == 0) ? 2 : 1;
-  ap.npairs = ap.rep / ap.nh;
-  ap.T = g.T;
-  ap.N = g.N;
-  ap.Pt = g.Pt;
-  ap.L = g.L;
-  ap.W = g.W;
-  ap.H = g.H;
-  ap.window_half = g.window / 2;
-  ap.tile_aligned = (mode != KREA_MODE_SCANLINE) || g.tile_aligned;
-  ap.n_tiles = g.n_tiles;
-  ap.q_lo = p->q_start;
-  ap.q_hi = p->q_start + q_len;
-  // logical tiles holding the slice's first and last physical rows
-  auto slot_of = [&](int t) { return t < g.T ? t : t - g.T + g.Pt; };
-  const int t_first = slot_of(ap.q_lo) / kTile, t_last = slot_of(ap.q_hi - 1) / kTile;
-  ap.tile_begin = t_first;
-  ap.n_slice_tiles = t_last - t_first + 1;
-  // Scanline: text query rows see every key tile, image rows only the text and their
-  // window, so the text tiles' CTAs go first and no long row starts in the last wave.
-  {
-    const int text_tiles = (g.T + kTile - 1) / kTile;
-    ap.n_heavy = mode == KREA_MODE_SCANLINE
-                     ? std::max(0, std::min(ap.tile_begin + ap.n_slice_tiles, text_tiles) - ap.tile_begin)
-                     : 0;
-  }
-  ap.nt_scale = (g.L + kTile - 1) / kTile;
-  const float scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt((float)d);
-  ap.scale_log2 = scale * 1.4426950408889634f;
-  ap.has_gate = gate != nullptr;
-  ap.out_f32 = p->out_dtype == KREA_F32;
-  ap.tma_out = tma_out ? 1 : 0;
-  ap.wait_limit = p->debug_wait_limit > 0 ? p->debug_wait_limit : (long long)2000000000LL;
-  ap.debug_flags = p->debug_flags;
-  if (p->lse && (reinterpret_cast<uintptr_t>(p->lse) & 3)) return KREA_ERR_INVALID_ARG;
-  ap.lse = p->lse;
-  return launch_attention(ap, maps, bf16, stream);
+  return launch_forward(q, k, v, gate, out, g, p, q_len, map.d_row_ptr, map.d_entries, map.n_int8 > 0,
+                        p->workspace, p->workspace_bytes, stream);
 }
 
 size_t krea_attn_bwd_scratch_bytes(int text_len, int grid_h, int grid_w, const krea_attn_params_t* p) {

@@ -45,6 +45,10 @@ struct HostMap {
 // stderr unless `quiet` (a size query).
 int build_map(const Geometry& g, HostMap* out, bool quiet = false);
 
+// Number of INT8 tiles of a TileMix map, counted in closed form per query tile
+// (no map is built); 0 for other modes. build_map checks its maps against it.
+long tilemix_int8_tiles(const Geometry& g);
+
 // Builds the map on the device (mapgen.cu): row_ptr[n_tiles + 1], and either packed
 // entries ((key tile << 2) | kind, packed != nullptr) or col / kind arrays. Nothing
 // is written past `capacity` entries; an overflow is reported through `status`.
@@ -117,6 +121,20 @@ struct BwdPrepParams {
 };
 int launch_bwd_prep(const BwdPrepParams& p, bool bf16, bool out32, void* stream);
 int launch_backward(const BwdDevParams& p, const BwdMaps& m, bool bf16, void* stream);
+
+// Pieces of a forward call shared by krea_attn_fwd and krea_attn_fwd_noalloc (api.cpp):
+// the params struct's own fields, the current device (sm_100), and the pointers,
+// alignment, strides and query slice of one call (writes the slice length).
+int check_params(const krea_attn_params_t* p);
+int check_device_sm100();
+int check_forward(const void* q, const void* k, const void* v, const void* gate, const void* out,
+                  const Geometry& g, const krea_attn_params_t* p, int* q_len);
+// Everything after the tile map: the TileMix quantiser into `workspace` (when
+// use_int8 or smooth_k), TMA descriptors, kernel parameters and the attention
+// launch, with the map's device row pointers and packed entries.
+int launch_forward(const void* q, const void* k, const void* v, const void* gate, void* out, const Geometry& g,
+                   const krea_attn_params_t* p, int q_len, const int32_t* row_ptr, const int32_t* entries,
+                   bool use_int8, void* workspace, size_t workspace_bytes, void* stream);
 
 // Resolves and validates the geometry of a call.
 int make_geometry(int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* p,

@@ -201,6 +201,18 @@ void log_map(const Geometry& g, const HostMap& m) {
 
 }  // namespace
 
+long tilemix_int8_tiles(const Geometry& g) {
+  if (g.mode != KREA_MODE_TILEMIX || g.pattern == KREA_PATTERN_ZERO) return 0;
+  const int nt = g.n_tiles, t0 = ceil_div(g.T, kTile);  // tiles holding a text token come first
+  long total = 0;
+  for (int a = t0; a < nt; ++a) {
+    // off-band image key tiles left and right of the diagonal
+    const long n = std::max(0, a - g.band_blocks - t0) + std::max(0, nt - 1 - a - g.band_blocks);
+    total += g.pattern == KREA_PATTERN_ONE ? n : (long)std::floor((double)g.percentage * (double)n + 0.5);
+  }
+  return total;
+}
+
 int build_map(const Geometry& g, HostMap* out, bool quiet) {
   if (!out) return KREA_ERR_INVALID_ARG;
   out->row_ptr.clear();
@@ -213,6 +225,8 @@ int build_map(const Geometry& g, HostMap* out, bool quiet) {
     case KREA_MODE_TILEMIX: build_tilemix(g, out); break;
     default: build_dense(g, out); break;
   }
+  // the closed-form count that callers without a host map rely on must agree
+  if (out->n_int8 != tilemix_int8_tiles(g)) return KREA_ERR_INVALID_ARG;
   if (!quiet && log_enabled()) log_map(g, *out);
   return KREA_OK;
 }

@@ -307,17 +307,20 @@ KREA_API int krea_attn_quantize(const void* q, const void* k, int text_len, int 
  * memory while they run (an arena or pool that forbids cudaMalloc/cudaFree, which
  * synchronise the device; a host framework that owns all device memory; a serving
  * loop that must not block on the allocator). It allocates, caches and frees
- * nothing: the tile map and the TileMix workspace live in one fixed 64 MiB array
- * in device memory declared by the library, held on every GPU that loads the
- * library until the process exits; params->workspace is ignored. Shapes whose
- * map plus workspace exceed 64 MiB return KREA_ERR_TOO_LARGE before any launch
- * (a 48/12-head TileMix call fits up to about 1 MP; dense and scanline calls fit
- * far beyond 4 MP). All calls share the array, so calls whose GPU work overlaps
- * (two streams, or two threads on one device) race and must not be issued; calls
- * on one stream are ordered. Each call rewrites everything it reads, nothing
- * needs clearing. The first call on a device looks up the array's device address;
- * make it before any CUDA graph capture on that device. The pages describe no
- * counterpart of this entry point. */
+ * nothing and copies nothing from the host: the tile map is built on `stream` by
+ * the device map builder (the same map krea_attn_fwd caches, bit for bit) and,
+ * with the TileMix workspace, lives in one fixed 64 MiB array in device memory
+ * declared by the library, held on every GPU that loads the library until the
+ * process exits; params->workspace is ignored. Results equal krea_attn_fwd's bit
+ * for bit. Shapes whose map (4 (n_tiles + 1) + 4 n_tiles^2 bytes) plus workspace
+ * exceed 64 MiB return KREA_ERR_TOO_LARGE before any launch (a 48/12-head TileMix
+ * call fits up to about 1 MP; dense and scanline calls fit far beyond 4 MP). All
+ * calls share the array, so calls whose GPU work overlaps (two streams, or two
+ * threads on one device) race and must not be issued; calls on one stream are
+ * ordered. Each call rewrites everything it reads, nothing needs clearing. The
+ * first call on a device looks up the array's device address; make it before any
+ * CUDA stream capture on that device. The pages describe no counterpart of this
+ * entry point. */
 KREA_API int krea_attn_fwd_noalloc(const void* q, const void* k, const void* v, const void* gate, void* out,
                                    int text_len, int grid_h, int grid_w, int mode,
                                    const krea_attn_params_t* params, void* stream);

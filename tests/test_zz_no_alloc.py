@@ -18,7 +18,6 @@ from synth import inputs as S
 
 pytestmark = pytest.mark.gpu
 
-TOL = 5e-4  # the tests' fp16 / fp32-accumulate bound; the same kernels run, so results agree far closer
 SCRATCH_BYTES = 64 << 20
 
 
@@ -61,20 +60,59 @@ CASES = [
            gate=True),
     S.Case("na_tilemix_again", 1, 8, 2, 128, 300, 25, 33, dtype="bf16", mode="tilemix", seed=43,
            qk_dist="normal_koffset", pattern="one", band_blocks=2),
+    S.Case("na_dense", 1, 4, 1, 64, 16, 8, 8, dtype="f16", mode="dense", seed=45, gate=True),
 ]
 
 
 def test_noalloc_matches_fwd_call_after_call():
+    # The same kernels on the same inputs, with the tile map built into the array by
+    # the device builder (bit-identical to the cached host map) and the TileMix
+    # workspace in the array: the outputs equal krea_attn_fwd's bit for bit, on two
+    # calls in a row of every case (consecutive calls share the array; each must
+    # stand on its own). params.workspace stays NULL throughout, TileMix included.
     dev = torch.device("cuda:0")
-    for case in CASES:  # consecutive calls share the array; each must stand on its own
+    for case in CASES:
         q, k, v, g = (t.to(dev) if t is not None else None for t in S.make_inputs(case))
         ref = reference_call(case, q, k, v, g)
-        rc, out, status = noalloc(case, q, k, v, g)
-        torch.cuda.synchronize()
-        assert rc == 0, K._lib.lib().krea_attn_error_string(rc)
-        assert int(status.item()) == 0
-        err = float((out - ref).abs().max())
-        assert err <= TOL, f"{case.name}: {err}"
+        for _ in range(2):
+            rc, out, status = noalloc(case, q, k, v, g)
+            torch.cuda.synchronize()
+            assert rc == 0, K._lib.lib().krea_attn_error_string(rc)
+            assert int(status.item()) == 0
+            assert torch.equal(out, ref), f"{case.name}: max |diff| {float((out - ref).abs().max())}"
+
+
+def test_noalloc_allocates_nothing():
+    # Once the kernels are loaded (a first call of each kind), further calls leave
+    # both torch's allocator and the device's free memory exactly where they were.
+    dev = torch.device("cuda:0")
+    inputs = []
+    for case in CASES:
+        q, k, v, g = (t.to(dev) if t is not None else None for t in S.make_inputs(case))
+        out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        p = _params(case, q, k, v, g, out, status)
+        assert not p.workspace  # no caller workspace, TileMix included
+        inputs.append((case, q, k, v, g, out, status, p))
+
+    def run_all():
+        for case, q, k, v, g, out, status, p in inputs:
+            rc = _lib.lib().krea_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                  g.data_ptr() if g is not None else None, out.data_ptr(),
+                                                  case.text_len, case.grid_h, case.grid_w, _lib.MODE[case.mode],
+                                                  ctypes.byref(p), torch.cuda.current_stream().cuda_stream)
+            assert rc == 0, K._lib.lib().krea_attn_error_string(rc)
+
+    run_all()
+    torch.cuda.synchronize()
+    torch_before = torch.cuda.memory_allocated(dev)
+    free_before, _ = torch.cuda.mem_get_info(dev)
+    for _ in range(3):
+        run_all()
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated(dev) == torch_before
+    assert torch.cuda.mem_get_info(dev)[0] == free_before
+    assert all(int(x[6].item()) == 0 for x in inputs)
 
 
 def test_noalloc_refuses_shapes_beyond_its_array():
