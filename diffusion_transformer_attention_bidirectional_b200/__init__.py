@@ -17,8 +17,8 @@ import torch
 from . import _lib
 from ._lib import KreaError, Params, check, lib
 
-__all__ = ["attention", "quantize", "get_map", "map_size", "workspace_bytes", "workspace_layout",
-           "make_params", "clear_cache", "KreaError"]
+__all__ = ["attention", "attention_backward", "quantize", "get_map", "map_size", "workspace_bytes",
+           "workspace_layout", "bwd_scratch_bytes", "make_params", "clear_cache", "KreaError"]
 
 _TORCH_DT = {torch.float16: "f16", torch.bfloat16: "bf16", torch.float32: "f32"}
 
@@ -65,6 +65,11 @@ def _stream_ptr(stream: Optional[torch.cuda.Stream], device: torch.device) -> in
 
 def workspace_bytes(mode: str, text_len: int, grid_h: int, grid_w: int, params: Params) -> int:
     return int(lib().krea_attn_workspace_bytes(text_len, grid_h, grid_w, _lib.MODE[mode], ctypes.byref(params)))
+
+
+def bwd_scratch_bytes(text_len: int, grid_h: int, grid_w: int, params: Params) -> int:
+    """Bytes of device scratch krea_attn_bwd needs for this geometry and params."""
+    return int(lib().krea_attn_bwd_scratch_bytes(text_len, grid_h, grid_w, ctypes.byref(params)))
 
 
 def workspace_layout(text_len: int, grid_h: int, grid_w: int, params: Params) -> dict:
@@ -116,13 +121,12 @@ def get_map_device(mode: str, text_len: int, grid_h: int, grid_w: int, params: O
 
 
 def rope_positions(text_len: int, grid_h: int, grid_w: int, device=None) -> torch.Tensor:
-    """[L, 3] int32 rotary positions: text token t at (t, 0, 0), image token (r, c) at (0, r, c)."""
+    """[L, 3] int32 rotary positions of the joint sequence, from krea_attn_rope_positions
+    (host work in the library), moved to `device` when given."""
     L = text_len + grid_h * grid_w
-    pos = torch.zeros(L, 3, dtype=torch.int32)
-    pos[:text_len, 0] = torch.arange(text_len, dtype=torch.int32)
-    img = torch.arange(grid_h * grid_w, dtype=torch.int32)
-    pos[text_len:, 1] = img // max(grid_w, 1)
-    pos[text_len:, 2] = img % max(grid_w, 1)
+    pos = torch.zeros(max(L, 1), 3, dtype=torch.int32)
+    check(lib().krea_attn_rope_positions(text_len, grid_h, grid_w, pos.data_ptr(), pos.shape[0]),
+          "rope_positions")
     return pos.to(device) if device is not None else pos
 
 
@@ -234,10 +238,13 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[
 def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[torch.Tensor],
                        out: torch.Tensor, dout: torch.Tensor, lse: torch.Tensor, *, text_len: int, grid_h: int,
                        grid_w: int, mode: str = "dense", stream: Optional[torch.cuda.Stream] = None,
-                       status: Optional[torch.Tensor] = None, **opts):
+                       status: Optional[torch.Tensor] = None, scratch: Optional[torch.Tensor] = None,
+                       grads: Optional[tuple] = None, **opts):
     """(dq, dk, dv, dgate) of krea_attn_fwd's output (fp32 tensors; dgate None without
     a gate). out, dout: the forward's output and its gradient, contiguous, same dtype;
-    lse: the forward's [B, Hq, L] log-sum-exp (attention(..., lse=...))."""
+    lse: the forward's [B, Hq, L] log-sum-exp (attention(..., lse=...)).
+    scratch (krea_attn_bwd_scratch_bytes bytes, uint8) and grads (dq, dk, dv, dgate:
+    contiguous fp32 tensors) may be passed in to reuse memory across calls."""
     _check_inputs(q, k, v, gate, out, dout, lse, status)
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -251,12 +258,26 @@ def attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: 
     if status is not None:
         p.status = status.data_ptr()
     out, dout = out.contiguous(), dout.contiguous()
-    dq = torch.empty(B, L, Hq, d, dtype=torch.float32, device=q.device)
-    dk = torch.empty(B, L, Hkv, d, dtype=torch.float32, device=q.device)
-    dv = torch.empty(B, L, Hkv, d, dtype=torch.float32, device=q.device)
-    dgate = torch.empty(B, L, Hq, d, dtype=torch.float32, device=q.device) if gate is not None else None
-    scratch = torch.empty(int(lib().krea_attn_bwd_scratch_bytes(text_len, grid_h, grid_w, ctypes.byref(p))),
-                          dtype=torch.uint8, device=q.device)
+    if grads is not None:
+        dq, dk, dv, dgate = grads
+        _check_inputs(dq, dk, dv, dgate)
+        for t, shape in ((dq, (B, L, Hq, d)), (dk, (B, L, Hkv, d)), (dv, (B, L, Hkv, d)), (dgate, (B, L, Hq, d))):
+            if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != shape):
+                raise ValueError("grads must be contiguous float32 tensors of the gradient shapes")
+        if gate is None:
+            dgate = None
+    else:
+        dq = torch.empty(B, L, Hq, d, dtype=torch.float32, device=q.device)
+        dk = torch.empty(B, L, Hkv, d, dtype=torch.float32, device=q.device)
+        dv = torch.empty(B, L, Hkv, d, dtype=torch.float32, device=q.device)
+        dgate = torch.empty(B, L, Hq, d, dtype=torch.float32, device=q.device) if gate is not None else None
+    need = bwd_scratch_bytes(text_len, grid_h, grid_w, p)
+    if scratch is None:
+        scratch = torch.empty(need, dtype=torch.uint8, device=q.device)
+    else:
+        _check_inputs(scratch)
+        if scratch.numel() * scratch.element_size() < need:
+            raise ValueError(f"scratch holds {scratch.numel() * scratch.element_size()} bytes, {need} needed")
     check(lib().krea_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                               gate.data_ptr() if gate is not None else None, out.data_ptr(), dout.data_ptr(),
                               lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),

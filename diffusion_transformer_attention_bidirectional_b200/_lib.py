@@ -114,6 +114,7 @@ SIGNATURES = {
     "krea_attn_default_rope": (None, [ctypes.POINTER(RopeParams), _I]),
     "krea_attn_bwd_scratch_bytes": (ctypes.c_size_t, [_I, _I, _I, _P]),
     "krea_attn_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _P, _VP]),
+    "krea_attn_rope_positions": (_I, [_I, _I, _I, _VP, ctypes.c_int32]),
     "krea_attn_rope_table": (_I, [_VP, _I, ctypes.POINTER(RopeParams), _VP, _VP]),
     "krea_attn_qk_prologue": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int64),
                                    ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(RopeParams), _VP, _VP, _VP]),

@@ -507,6 +507,24 @@ int check_rope(const krea_rope_params_t* r, int head_dim) {
 }
 }  // namespace
 
+int krea_attn_rope_positions(int text_len, int grid_h, int grid_w, int32_t* pos, int32_t capacity) {
+  if (!pos || text_len < 0 || grid_h < 0 || grid_w < 0 || (grid_h == 0) != (grid_w == 0)) return KREA_ERR_INVALID_ARG;
+  const long long L = (long long)text_len + (long long)grid_h * grid_w;
+  if (L <= 0 || L > (1LL << 24) || capacity < L) return KREA_ERR_INVALID_ARG;
+  for (int t = 0; t < text_len; ++t) {
+    pos[3 * t] = t;
+    pos[3 * t + 1] = 0;
+    pos[3 * t + 2] = 0;
+  }
+  for (int r = 0, i = text_len; r < grid_h; ++r)
+    for (int c = 0; c < grid_w; ++c, ++i) {
+      pos[3 * i] = 0;
+      pos[3 * i + 1] = r;
+      pos[3 * i + 2] = c;
+    }
+  return KREA_OK;
+}
+
 int krea_attn_rope_table(const int32_t* pos, int tokens, const krea_rope_params_t* rope, float* table,
                          void* stream) {
   int rc = check_rope(rope, 0);

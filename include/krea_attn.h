@@ -136,7 +136,12 @@ KREA_API int krea_attn_fwd(const void* q, const void* k, const void* v, const vo
                   int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* params,
                   void* stream);
 
-/* Bytes of caller-allocated workspace krea_attn_fwd needs (0 if none). */
+/* Bytes of caller-allocated workspace krea_attn_fwd needs (0 if none): only TileMix
+ * calls need any, for the smooth_k centred keys ("Krea 2 TileMix Attention (FP16/INT8
+ * tiles)", section "The inputs that matter") and the INT8 codes and block scales of
+ * the tiles the map sends to INT8 (section "What it actually patches"; the
+ * per-(batch, head, 128-token block) absmax/127 scheme is this library's, the pages
+ * give none). Returns 0 for other modes or invalid params; pure host arithmetic. */
 KREA_API size_t krea_attn_workspace_bytes(int text_len, int grid_h, int grid_w, int mode,
                                  const krea_attn_params_t* params);
 
@@ -152,13 +157,23 @@ KREA_API int krea_attn_workspace_layout(int text_len, int grid_h, int grid_w, in
                                const krea_attn_params_t* params, krea_attn_ws_layout_t* out);
 
 /* Size of the tile map: *n_tiles query tiles (the logical sequence, text slot
- * included for scanline) and *nnz listed (query tile, key tile) pairs. */
+ * included for scanline) and *nnz listed (query tile, key tile) pairs. The map is
+ * the 128-tile block map of "Krea 2 Scanline Attention", section "What the mask
+ * actually is" (scanline), or the per-tile FP16/INT8 routing of "Krea 2 TileMix
+ * Attention (FP16/INT8 tiles)", sections "What it actually patches" and "The inputs
+ * that matter" (TileMix); dense lists every pair. Host work; needs no GPU;
+ * KREA_ERR_INVALID_ARG for a bad geometry or params. */
 KREA_API int krea_attn_map_size(int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* params,
                        int32_t* n_tiles, int32_t* nnz);
 
 /* Copy the tile map into HOST buffers: row_ptr[n_tiles + 1], col[nnz] (key tiles,
  * ascending per row) and kind[nnz] (KREA_KIND_* bits). `capacity` is the length of
- * col and kind. Pure host work; needs no GPU. */
+ * col and kind (KREA_ERR_INVALID_ARG when smaller than nnz, or a NULL buffer). The
+ * map rules are those of krea_attn_map_size: the scanline block map ("Krea 2
+ * Scanline Attention", section "What the mask actually is") or TileMix's per-tile
+ * routing ("Krea 2 TileMix Attention (FP16/INT8 tiles)", sections "What it actually
+ * patches" and "The inputs that matter"). The caller owns the buffers; pure host
+ * work, needs no GPU. */
 KREA_API int krea_attn_get_map(int text_len, int grid_h, int grid_w, int mode, const krea_attn_params_t* params,
                       int32_t* row_ptr, int32_t* col, uint8_t* kind, int32_t capacity);
 
@@ -192,6 +207,17 @@ typedef struct {
 
 /* (head_dim/4, 3 head_dim/8, 3 head_dim/8) channels, theta 10000, eps 1e-6. */
 KREA_API void krea_attn_default_rope(krea_rope_params_t* rope, int head_dim);
+
+/* Rotary positions of the joint [text, image] sequence, the layout this library
+ * takes for the 3-axis RoPE the pages name ("Krea 2 TileMix Attention (FP16/INT8
+ * tiles)", section "What it actually patches": QK RMSNorm and 3-axis RoPE run right
+ * before the core; the pages give no layout): text token t at (t, 0, 0), image token
+ * at grid row r, column c at (0, r, c), image tokens row-major after the text.
+ * Writes pos[L][3] int32 (L = text_len + grid_h * grid_w) into a HOST buffer of
+ * `capacity` rows; KREA_ERR_INVALID_ARG for a bad geometry, a NULL pointer or
+ * capacity < L. Pure host work; needs no GPU. Other layouts are passed to
+ * krea_attn_rope_table directly. */
+KREA_API int krea_attn_rope_positions(int text_len, int grid_h, int grid_w, int32_t* pos, int32_t capacity);
 
 /* Rotary table of a geometry: table[t][j] = (cos, sin) of pair j's angle for
  * token t (pairs numbered axis by axis), from pos [tokens][3] int32 (device),
@@ -298,8 +324,16 @@ KREA_API int krea_attn_ipc_free(void* ptr);
 KREA_API int krea_attn_ipc_open(const void* handle, void** ptr);
 KREA_API int krea_attn_ipc_close(void* ptr);
 
-/* Run only the TileMix quantiser (key mean, centred keys, INT8 codes and scales)
- * into params->workspace, laid out as krea_attn_workspace_layout() says. */
+/* Run only the TileMix quantiser into params->workspace (device memory of
+ * krea_attn_workspace_bytes() bytes, 16-byte aligned, owned by the caller), laid out
+ * as krea_attn_workspace_layout() says: the key mean per (batch, kv head, channel)
+ * and the centred keys k - mean (smooth_k: "Krea 2 TileMix Attention (FP16/INT8
+ * tiles)", section "The inputs that matter"), then the symmetric INT8 codes and
+ * absmax/127 scales of q and of the (centred) keys per (batch, head, 128-token
+ * block), the scheme this library fixes (the pages give none). q, k: device
+ * tensors as for krea_attn_fwd; head_dim 128. Asynchronous on `stream`. Errors:
+ * KREA_ERR_INVALID_ARG (pointers, strides, geometry), KREA_ERR_UNSUPPORTED
+ * (head_dim), KREA_ERR_WORKSPACE, KREA_ERR_NO_DEVICE, KREA_ERR_CUDA. */
 KREA_API int krea_attn_quantize(const void* q, const void* k, int text_len, int grid_h, int grid_w,
                        const krea_attn_params_t* params, void* stream);
 
@@ -347,7 +381,10 @@ KREA_API int krea_attn_bwd(const void* q, const void* k, const void* v, const vo
 /* Release every cached tile map on every device. */
 KREA_API void krea_attn_clear_cache(void);
 
-/* Static text for a krea_status_t. */
+/* Static text for a krea_status_t (never NULL; "unknown error" for other codes).
+ * The codes replace the pages' silent dense fallbacks ("Krea 2 TileMix Attention
+ * (FP16/INT8 tiles)", section "Where people get burned"): an unsupported input is
+ * an error, never a different computation. */
 KREA_API const char* krea_attn_error_string(int code);
 
 /* KREA_ATTN_ABI_VERSION of the loaded library. */

@@ -8,6 +8,7 @@ import re
 import subprocess
 import tempfile
 
+import numpy as np
 import pytest
 import torch
 
@@ -133,6 +134,11 @@ def test_prologue_arguments_rejected_without_gpu():
 def test_rope_positions_layout():
     pos = K.rope_positions(2, 2, 3)
     assert pos.tolist() == [[0, 0, 0], [1, 0, 0], [0, 0, 0], [0, 0, 1], [0, 0, 2], [0, 1, 0], [0, 1, 1], [0, 1, 2]]
+    buf = np.zeros((7, 3), dtype=np.int32)
+    L = _lib.lib()
+    assert L.krea_attn_rope_positions(2, 2, 3, buf.ctypes.data, 7) == _lib.ERR_INVALID_ARG  # capacity < L
+    assert L.krea_attn_rope_positions(2, 2, 0, buf.ctypes.data, 7) == _lib.ERR_INVALID_ARG  # half a grid
+    assert L.krea_attn_rope_positions(2, 2, 3, None, 8) == _lib.ERR_INVALID_ARG
 
 
 def test_exchange_layout_matches_header():
