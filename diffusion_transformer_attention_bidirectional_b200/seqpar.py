@@ -216,6 +216,11 @@ class SequenceParallelAttention:
     # how buffers other ranks map are made and opened (CUDA IPC)
     buffer_cls = PeerBuffer
     mapping_cls = PeerMapping
+    # Process-group backends whose all-reduce orders the ranks' device work: NCCL
+    # runs it on the current CUDA stream, so every rank's stores into peer buffers
+    # issued before it have completed when work after it starts. Other backends
+    # give no such ordering on the stream; world > 1 refuses them.
+    barrier_backends = ("nccl",)
 
     def __init__(self, batch: int, tokens_per_rank: int, q_heads: int, kv_heads: int, head_dim: int,
                  dtype: torch.dtype = torch.bfloat16, out_dtype: torch.dtype = torch.float32, group=None,
@@ -245,6 +250,11 @@ class SequenceParallelAttention:
                 self.dests[name] = Destinations.of([self.local[name]])
             self.o_heads = torch.empty((batch, L, q_heads, head_dim), dtype=out_dtype, device=device)
             return
+        backend = dist.get_backend(group)
+        if backend not in self.barrier_backends:
+            raise RuntimeError(f"SequenceParallelAttention over {W} ranks needs a process group whose "
+                               f"collectives are ordered on the CUDA stream ({', '.join(self.barrier_backends)}); "
+                               f"got {backend}")
         own = {name: self.buffer_cls(shape, dt) for name, (shape, dt) in shapes.items()}
         self._keep.append(own)
         handles = {name: b.handle_bytes() for name, b in own.items()}

@@ -229,6 +229,15 @@ def _sequence_parallel_class_worker(rank, world, port, shared_dir, results):
         seqpar._core = fake_core
         seqpar.SequenceParallelAttention.buffer_cls = FileBuffer
         seqpar.SequenceParallelAttention.mapping_cls = FileMapping
+        # a gloo group is refused on the real path (its all-reduce is not ordered
+        # on a CUDA stream); here every buffer is host memory, so it orders them
+        try:
+            seqpar.SequenceParallelAttention(1, Ls, case.q_heads, case.kv_heads, case.head_dim,
+                                             dtype=torch.float64, out_dtype=torch.float64, device="cpu")
+            raise AssertionError("a gloo group was accepted")
+        except RuntimeError as e:
+            assert "ordered on the CUDA stream" in str(e)
+        seqpar.SequenceParallelAttention.barrier_backends = ("gloo",)
 
         spa = seqpar.SequenceParallelAttention(1, Ls, case.q_heads, case.kv_heads, case.head_dim,
                                                dtype=torch.float64, out_dtype=torch.float64, device="cpu")
