@@ -85,6 +85,10 @@ constexpr long long kDrainLimit = 4000000000LL;
 // then bound by issue and latency rather than by the exponential unit; the
 // polynomial stays available (debug_flags bit 1 runs every exponential on it).
 constexpr uint32_t kPolyMask = 0x00u;
+// bf16 query tiles whose map row lists at most this many key tiles (<= 1024 keys)
+// take P to 16 bits: the 2^-9 relative rounding of single weights bounds the
+// error of short rows near 2^-9 max|v|, and only averages out over longer rows.
+constexpr int kSplitMaxTiles = 8;
 constexpr float kNegInf = -INFINITY;
 
 struct Ctl {
@@ -214,7 +218,11 @@ __device__ __forceinline__ float i2f_exact(uint32_t x) {
 // (keys 0..63) on half_bar before the exponentials of keys 64..127 are taken, so
 // that PV on those keys overlaps them; updates m, l and, when the running maximum
 // moves, rescales O in TMEM (before either half of P is released).
-template <bool BF16, bool IS8, bool MASKED, bool ALL_POLY>
+// SPLIT (bf16 only): each weight p is also written as a second bf16 term
+// p - bf16(p) over columns 64..127 of S (free once the row is in registers), so
+// that two PV products give P to 16 significant bits instead of 8 (rows with few
+// admitted keys, where the rounding of single weights does not average out).
+template <bool BF16, bool IS8, bool MASKED, bool ALL_POLY, bool SPLIT>
 __device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int a1, int a2, int a3, float& m,
                                              float& l, bool first, uint32_t tS, uint32_t tO, int d,
                                              uint32_t half_bar) {
@@ -276,8 +284,13 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int
       if (i & 1) acc1 = ptx::add2(acc1, ptx::f2(p0, p1));
       else acc0 = ptx::add2(acc0, ptx::f2(p0, p1));
       pk[i] = pack2<BF16>(p0, p1);
+      if constexpr (SPLIT) {  // the rounding residual, itself rounded to bf16
+        const float r0 = p0 - __uint_as_float(pk[i] << 16), r1 = p1 - __uint_as_float(pk[i] & 0xffff0000u);
+        v[64 * h + i] = pack2<BF16>(r0, r1);  // keys 64h .. 64h+63 of v are consumed: reuse their registers
+      }
     }
     ptx::tmem_st32(tS + 32u * h, pk);
+    if constexpr (SPLIT) ptx::tmem_st32(tS + 64u + 32u * h, *reinterpret_cast<const uint32_t(*)[32]>(&v[64 * h]));
     if (h == 0) {  // keys 0..63 of P are in TMEM: the tensor core may start on them
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -298,7 +311,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int
 // completes every 64 cycles).
 template <bool BF16, int D>
 __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base, uint32_t tmem, int e0, int n,
-                                           int nh, const Ctl& ctl) {
+                                           int nh, const Ctl& ctl, bool split) {
   auto bar = [&](int i) { return base + SM_BAR + 8u * (uint32_t)i; };
   constexpr uint32_t ab = BF16 ? 1u : 0u;
   constexpr uint32_t ID_QK = ptx::idesc(1, ab, 0, 0, 128, 128);
@@ -327,10 +340,11 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
       }
     }
   };
-  // PV over keys 64 half .. 64 half + 63 of the tile
-  auto pv = [&](int i, uint32_t slot, int half, uint32_t acc) {
+  // PV over keys 64 half .. 64 half + 63 of the tile; lo = 1: the bf16 residual
+  // terms of P (columns 64..127 of S) instead of the rounded weights
+  auto pv = [&](int i, uint32_t slot, int half, uint32_t acc, int lo = 0) {
     const uint32_t dO = tmem + 256u + (uint32_t)i * 128u;
-    const uint32_t aP = tmem + (uint32_t)i * 128u + 32u * (uint32_t)half;
+    const uint32_t aP = tmem + (uint32_t)i * 128u + 64u * (uint32_t)lo + 32u * (uint32_t)half;
     const uint32_t vd = dv + slot * (kTileBytes >> 4) + 512u * (uint32_t)half;  // 64 rows x 128 B
     ptx::mma_f16_ts_lo(dO, aP, vd, ID_PV, acc);
 #pragma unroll
@@ -382,6 +396,10 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
         if (!ok) break;
         ptx::tc_fence_after();
         pv(i, slot_v, 1, 1u);
+        if (split) {
+          pv(i, slot_v, 0, 1u, 1);
+          pv(i, slot_v, 1, 1u, 1);
+        }
         if (has_next) {
           if (i == 0) {
             ok = wait1(ctl, bar(BAR_FULL + slot_k), (it / kSlots) & 1) && need_q8(kind_next);
@@ -490,6 +508,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // no text padding inside the tile; rows past L are clipped by the TMA unit.
   const int qrow0 = tile_row0(qt, p);
   const int s0q = qt * kTile;
+  // bf16 rows with at most kSplitMaxTiles key tiles: P to 16 bits (two PV terms)
+  const bool split = BF16 && n <= kSplitMaxTiles;
   const bool staged = p.tma_out && ((s0q + kTile <= p.T) || (s0q >= p.Pt) || (p.T == p.Pt)) &&
                       qrow0 >= p.q_lo && min(qrow0 + kTile, p.L) <= p.q_hi;
 
@@ -555,8 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      if (d == 128) mma_thread<BF16, 128>(p, base, tmem, e0, n, nh, ctl);
-      else mma_thread<BF16, 64>(p, base, tmem, e0, n, nh, ctl);
+      if (d == 128) mma_thread<BF16, 128>(p, base, tmem, e0, n, nh, ctl, split);
+      else mma_thread<BF16, 64>(p, base, tmem, e0, n, nh, ctl, split);
     }
   } else if (warp == 10) {
     // ------------------------------------------------------------- INT8 query codes
@@ -620,10 +640,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s0 = kb * kTile;
         const int a1 = p.T - s0, a2 = klo - s0, a3 = khi - s0;
         const bool first = t == 0;
-        if (kind == 0) softmax_tile<BF16, false, false, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, bar(BAR_PH + wg));
-        else if (kind == 1) softmax_tile<BF16, false, true, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, bar(BAR_PH + wg));
-        else if (kind == 2) softmax_tile<BF16, true, false, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, bar(BAR_PH + wg));
-        else softmax_tile<BF16, true, true, ALL_POLY>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, bar(BAR_PH + wg));
+        const uint32_t hb = bar(BAR_PH + wg);
+        if (BF16 && split) {
+          if (kind == 0) softmax_tile<BF16, false, false, ALL_POLY, BF16>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, hb);
+          else if (kind == 1) softmax_tile<BF16, false, true, ALL_POLY, BF16>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, hb);
+          else if (kind == 2) softmax_tile<BF16, true, false, ALL_POLY, BF16>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, hb);
+          else softmax_tile<BF16, true, true, ALL_POLY, BF16>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, hb);
+        } else {
+          if (kind == 0) softmax_tile<BF16, false, false, ALL_POLY, false>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, hb);
+          else if (kind == 1) softmax_tile<BF16, false, true, ALL_POLY, false>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, hb);
+          else if (kind == 2) softmax_tile<BF16, true, false, ALL_POLY, false>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, hb);
+          else softmax_tile<BF16, true, true, ALL_POLY, false>(v, mult, a1, a2, a3, m, l, first, tS, tO, d, hb);
+        }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();

@@ -2,13 +2,15 @@
 
 Small cases are compared element by element on every output; the full-size
 workloads on sampled query tiles (whole 128-row tiles, several heads) that the
-oracle computes row by row. Tolerances (max |gpu - oracle|, outputs of unit
-scale): 8e-3 when INT8 tiles are present; 5e-4 for fp16 inputs and for the
-dense full-size workloads. The P operand of the PV product has the type of V, so with
-bf16 inputs every softmax weight w_j is rounded to 8 significant bits, relative
-error at most 2^-9, and |out - exact| <= 2^-9 * sum_j w_j |v_j| <= 2^-9 max_j |v_j|.
-Over a few dozen admitted keys that bound is reached (~2e-3); over thousands of
-keys the errors average out below 5e-4. Other bf16 cases use that bound.
+oracle computes row by row. Tolerances (max |gpu - oracle| on unit-scale
+outputs), the ones the specification states: 8e-3 when INT8 tiles are present;
+2e-3 for FP16 tiles; 5e-4 with fp32 QK accumulation (calls that set
+qk_fp32_accumulate) and for fp16 inputs. The P operand of the PV product has the
+type of V, so with bf16 inputs each softmax weight is rounded to 8 significant
+bits (relative error 2^-9); over the thousand-plus keys of a long row those
+errors average out well below 2e-3, and rows of at most eight key tiles carry P
+to 16 bits (a second bf16 term) so that short rows, where single weights
+dominate, stay inside the bound too. Every comparison prints its observed error.
 """
 import numpy as np
 import pytest
@@ -20,7 +22,8 @@ from synth import inputs as S
 
 pytestmark = pytest.mark.gpu
 
-TOL_FP = 5e-4
+TOL_FP = 5e-4     # fp32 QK accumulation, fp16 inputs
+TOL_FP16_TILES = 2e-3
 TOL_INT8 = 8e-3
 
 
@@ -49,8 +52,8 @@ def compare(case, out_gpu, q, k, v, g, rows=None, heads=None, tol=None):
     if tol is None:
         if case.mode == "tilemix" and case.pattern != "zero":
             tol = TOL_INT8
-        elif case.dtype == "bf16":
-            tol = max(TOL_FP, 2.0 ** -9 * float(v.float().abs().max()) + 1e-5)
+        elif case.dtype == "bf16" and not case.qk_fp32_accumulate:
+            tol = TOL_FP16_TILES
         else:
             tol = TOL_FP
     ref = ko.attention(case, q, k, v, g, rows=rows, heads=heads)["out"]
@@ -105,7 +108,7 @@ def test_batch_and_out_dtype():
     q, k, v, g = S.make_inputs(c)
     out = gpu_run(c, q, k, v, g, out_dtype=torch.bfloat16)
     assert out.dtype == torch.bfloat16
-    compare(c, out, q, k, v, g, tol=4e-3)  # bf16 output rounding (2^-9 relative)
+    compare(c, out, q, k, v, g, tol=4e-3)  # 2e-3 FP16-tile bound + 2^-9 rounding of the bf16 output
 
 
 def test_strided_inputs():

@@ -88,7 +88,7 @@ def test_prologue_then_attention_matches_oracle_chain():
     qo = torch.from_numpy(ko.qk_prologue(q, pos)).to(torch.bfloat16)
     ko_ = torch.from_numpy(ko.qk_prologue(k, pos)).to(torch.bfloat16)
     ref = ko.attention(c, qo, ko_, v, g)["out"]
-    vmax = float(np.max(np.abs(v.float().numpy())))
     err = float(np.max(np.abs(out.cpu().numpy() - ref)))
-    # bf16 P rounding bound, plus inputs that may differ from the oracle's by one ulp
-    assert err <= 2.0 ** -9 * vmax + 2e-3, err
+    print(f"[parity] prologue -> scanline attention chain: max |gpu - oracle| = {err:.3e} (tol 2e-3)")
+    # the FP16-tile bound; q and k may differ from the oracle's rounded values by one ulp
+    assert err <= 2e-3, err

@@ -6,12 +6,17 @@ running the ranks one after the other computes what concurrent ranks would.
 The result must equal the unsharded call bit for bit: the QK prologue of a row
 does not depend on which rank computes it, every head of the core is
 independent, and the TileMix key mean sums fixed 128-token chunks in fp64
-whatever the head count. The unsharded call is checked against the oracle by
-the other GPU tests; the decomposition itself is checked against the oracle
+whatever the head count. Each case also holds the exchanged result itself
+against the oracle's own chain (QK prologue, rounding to the input dtype,
+attention) on sampled rows at every shard's edges and middle, at the bounds the
+other parity tests use. The decomposition itself is checked against the oracle
 on CPU ranks in test_dist.py. Destinations start as NaN, so a row the exchange
 failed to write breaks the equality."""
+import numpy as np
 import pytest
 import torch
+
+from oracle import krea_oracle as ko
 
 import diffusion_transformer_attention_bidirectional_b200 as K
 from diffusion_transformer_attention_bidirectional_b200 import seqpar
@@ -82,6 +87,33 @@ def run_case(c, world, pad_heads=0, out_dtype=torch.float32):
     ref = K.attention(qn, kn, v, g, **geo, **mode_opts(c))
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+    check_against_oracle(c, out, world, gq, gk)
+
+
+def check_against_oracle(c, out, world, gq, gk):
+    """The exchanged output on sampled rows (the first, middle and last rows of every
+    shard) and heads against the oracle's prologue -> attention chain."""
+    q, k, v, g = S.make_inputs(c)
+    L = c.seq_len
+    Ls = L // world
+    rows = sorted({t for r in range(world) for t in (r * Ls, r * Ls + 1, r * Ls + Ls // 2, (r + 1) * Ls - 1)})
+    Hq = q.shape[2]
+    heads = sorted({0, Hq // 2, Hq - 1})
+    pos = ko.rope_positions(c.text_len, c.grid_h, c.grid_w)
+    td = TDT[c.dtype]
+    qo = torch.from_numpy(ko.qk_prologue(q, pos, gamma=gq.cpu().numpy())).to(td)
+    ko_ = torch.from_numpy(ko.qk_prologue(k, pos, gamma=gk.cpu().numpy())).to(td)
+    want = ko.attention(c, qo, ko_, v, g, rows=rows, heads=heads)["out"][:, :, heads]
+    got = out.float().cpu().numpy()[:, rows][:, :, heads]
+    if c.mode == "tilemix" and c.pattern != "zero":
+        tol = 8e-3
+    elif out.dtype == torch.float16:
+        tol = 5e-4 + 2.0 ** -11  # fp16 output rounding of unit-scale values
+    else:
+        tol = 2e-3 if c.dtype == "bf16" else 5e-4
+    err = float(np.max(np.abs(got - want)))
+    print(f"[parity] exchange {c.name} over {world} ranks: max |gpu - oracle| = {err:.3e} (tol {tol:.1e})")
+    assert err <= tol * max(1.0, float(np.max(np.abs(want))))
 
 
 def test_scanline_1mp_over_four_ranks():
