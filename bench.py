@@ -25,6 +25,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 import numpy as np
@@ -182,53 +183,107 @@ def job_throughput(flops_per_rank: float, world: int, ms: float) -> float:
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
+    """SM clock and clock-event reasons sampled DURING the timed region. Reads only:
+    NVML queries from a background thread every ~10 ms (so that a timed region of
+    a fraction of a second still gets dozens of samples), else `nvidia-smi -lms`.
+    start() returns once the first sample is in."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, device_index: int):
-        self.idx = device_index
+    def __init__(self, device):
+        self.device = device
+        self.idx = device.index if device.index is not None else 0
         self.proc = None
         self.file = None
+        self.thread = None
+        self.samples = []  # (sm_mhz, max_mhz, set of reasons)
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+        except Exception:  # noqa: BLE001 - fall back to the ordinal
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.idx)
 
     def start(self):
         try:
-            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.file, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            nv, h = self._nvml_handle()
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.stop_flag = threading.Event()
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((sm, mx, {n for n, b in bits.items() if r & b}))
+                    except Exception:  # noqa: BLE001 - a failed read is a missing sample
+                        pass
+                    self.stop_flag.wait(0.01)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            self.source = "nvml"
+        except Exception:  # noqa: BLE001 - no NVML: nvidia-smi
+            try:
+                self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+                self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.QUERY}",
+                                              "--format=csv,noheader,nounits", "-lms", "50"],
+                                             stdout=self.file, stderr=subprocess.DEVNULL)
+                self.source = "nvidia-smi"
+            except (OSError, FileNotFoundError):
+                self.proc = None
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and not self._have_sample():
+            time.sleep(0.01)
+
+    def _have_sample(self):
+        if self.thread is not None:
+            return len(self.samples) > 0
+        if self.file is not None:
+            return os.path.getsize(self.file.name) > 0
+        return True
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.file.flush()
-        self.file.seek(0)
-        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
-        os.unlink(self.file.name)
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            if len(r) < 9:
-                continue
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            rows = list(self.samples)
+        elif self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(r[1]))
-                mx = max(mx, float(r[2]))
-            except ValueError:
-                continue
-            for name, val in zip(names, r[5:9]):
-                if "Active" in val and "Not" not in val:
-                    reasons.add(name)
-        if not sm:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.file.flush()
+            self.file.seek(0)
+            rows = []
+            for r in (x.split(",") for x in self.file.read().strip().splitlines() if x.strip()):
+                if len(r) < 9:
+                    continue
+                try:
+                    rows.append((float(r[1]), float(r[2]),
+                                 {n for n, v in zip(self.NAMES, r[5:9]) if "Active" in v and "Not" not in v}))
+                except ValueError:
+                    continue
+            os.unlink(self.file.name)
+        else:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not rows:
+            return None
+        reasons = set().union(*(r[2] for r in rows))
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "source": self.source}
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -412,7 +467,7 @@ def run_ours(args, rank, world, device):
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during warm-up")
 
-    sampler = ClockSampler(device.index if device.index is not None else 0)
+    sampler = ClockSampler(device)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)

@@ -68,8 +68,8 @@ constexpr int BAR_Q = 0, BAR_FULL = 1, BAR_EMPTY = BAR_FULL + kSlots, BAR_S = BA
               BAR_P = BAR_S + 2, BAR_O = BAR_P + 2, BAR_DRAIN = BAR_O + 2, BAR_NEVER = BAR_DRAIN + 1,
               BAR_QFREE = BAR_NEVER + 1,  // the last QK^T finished: the Q area may be reused
               BAR_GATE = BAR_QFREE + 1,   // gate tiles landed in the Q area
-              BAR_EPI = BAR_GATE + 1,     // 2: all 128 rows of head i staged for the TMA store
-              BAR_Q8 = BAR_EPI + 2,       // INT8 query codes landed (rows with INT8 tiles only)
+              BAR_EPI = BAR_GATE + 1,     // 2 x 4: box x of head i staged for its TMA store (i * 4 + x)
+              BAR_Q8 = BAR_EPI + 8,       // INT8 query codes landed (rows with INT8 tiles only)
               BAR_PH = BAR_Q8 + 1,        // 2: the first half of P_i (keys 0..63) written
               N_BARS = BAR_PH + 2;
 constexpr uint32_t SM_TMEM_PTR = SM_BAR + 8 * N_BARS;
@@ -78,6 +78,7 @@ constexpr uint32_t SMEM_USED = SM_BAR + 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // slack to align the base to 1024 bytes
 static_assert(8 * N_BARS + 8 <= 256, "barrier block overflow");
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+static_assert(kSlots == 4, "the staged epilogue places head 0's output in the even slots, head 1's in the odd");
 constexpr long long kDrainLimit = 4000000000LL;
 // Pairs of exponentials computed by the FMA-pipe polynomial: bit (i % 8) of
 // kPolyMask for pair i. Measured on B200 inside this kernel: every offload
@@ -147,6 +148,33 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ int tile_row0(int tile, const AttnDevParams& p) {
   const int s0 = tile * kTile;
   return s0 < p.Pt ? s0 : s0 - p.Pt + p.T;
+}
+
+// Work item of CTA idx: (batch, kv head, head pair, query tile), query tile
+// fastest; the slice's first n_heavy query tiles (the longest map rows) come
+// first for every (batch, kv head, head pair), then the rest.
+struct Item {
+  int qt, pair, g, b;
+};
+__device__ __forceinline__ Item decode_item(int idx, const AttnDevParams& p) {
+  const int heavy_ctas = p.B * p.Hkv * p.npairs * p.n_heavy;
+  int ql;
+  if (idx < heavy_ctas) {
+    ql = idx % p.n_heavy;
+    idx /= p.n_heavy;
+  } else {
+    idx -= heavy_ctas;
+    const int n_light = p.n_slice_tiles - p.n_heavy;
+    ql = p.n_heavy + idx % n_light;
+    idx /= n_light;
+  }
+  Item it;
+  it.qt = p.tile_begin + ql;
+  it.pair = idx % p.npairs;
+  idx /= p.npairs;
+  it.g = idx % p.Hkv;
+  it.b = idx / p.Hkv;
+  return it;
 }
 
 template <bool BF16>
@@ -356,6 +384,9 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
     for (int k = 1; k < 4; ++k)  // 16 keys per step: 8 TMEM columns of P, 16 rows of V (2 KB)
       ptx::mma_f16_ts_lo(dO, aP + 8u * k, vd + 128u * k, ID_PV, 1);
   };
+  // the first two map entries are read before any wait, so their latency hides behind Q's
+  const int ent0 = p.entries[e0];
+  int e_next = n > 1 ? p.entries[e0 + 1] : 0;  // map entries are read one tile ahead
   bool ok = wait1(ctl, bar(BAR_Q), 0);
   bool q8_ready = false;  // the INT8 query codes are awaited before the first INT8 tile
   auto need_q8 = [&](int kind) {
@@ -370,11 +401,10 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
     ptx::tc_fence_after();
     ok = wait1(ctl, bar(BAR_FULL + 0), 0);
   }
-  if (ok) ok = need_q8(p.entries[e0] & 3);
+  if (ok) ok = need_q8(ent0 & 3);
   if (ok) {
     ptx::tc_fence_after();
-    const int kind0 = p.entries[e0] & 3;
-    int e_next = n > 1 ? p.entries[e0 + 1] : 0;  // map entries are read one tile ahead
+    const int kind0 = ent0 & 3;
     for (int i = 0; i < nh; ++i) {
       qk(i, kind0, 0);
       ptx::tc_commit(bar(BAR_S + i));
@@ -405,6 +435,7 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
           pv(i, slot_v, 0, 1u, 1);
           pv(i, slot_v, 1, 1u, 1);
         }
+        if (!has_next) ptx::tc_commit(bar(BAR_O + i));  // O_i is final: its epilogue may start
         if (has_next) {
           if (i == 0) {
             ok = wait1(ctl, bar(BAR_FULL + slot_k), (it / kSlots) & 1) && need_q8(kind_next);
@@ -424,8 +455,6 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
       }
     }
   }
-  if (ok)
-    for (int i = 0; i < nh; ++i) ptx::tc_commit(bar(BAR_O + i));
   // every MMA this thread issued finishes before TMEM is freed, also when a
   // softmax warp gave up waiting on O
   ptx::tc_commit(bar(BAR_DRAIN));
@@ -441,26 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sb = smem_raw + (base - raw);
 
-  // work item: (batch, kv head, head pair, query tile), query tile fastest; the
-  // slice's first n_heavy query tiles (the longest map rows) come first for every
-  // (batch, kv head, head pair), then the rest
-  int idx = blockIdx.x;
-  const int heavy_ctas = p.B * p.Hkv * p.npairs * p.n_heavy;
-  int ql;
-  if (idx < heavy_ctas) {
-    ql = idx % p.n_heavy;
-    idx /= p.n_heavy;
-  } else {
-    idx -= heavy_ctas;
-    const int n_light = p.n_slice_tiles - p.n_heavy;
-    ql = p.n_heavy + idx % n_light;
-    idx /= n_light;
-  }
-  const int qt = p.tile_begin + ql;
-  const int pair = idx % p.npairs;
-  idx /= p.npairs;
-  const int g = idx % p.Hkv;
-  const int b = idx / p.Hkv;
+  const Item item = decode_item((int)blockIdx.x, p);
+  const int qt = item.qt, pair = item.pair, g = item.g, b = item.b;
   const int h0 = g * p.rep + pair * p.nh;
   const int e0 = p.row_ptr[qt];
   const int n = p.row_ptr[qt + 1] - e0;
@@ -492,8 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(bar(BAR_Q8), 1);
     ptx::mbar_init(bar(BAR_PH + 0), 4);  // one arrival per softmax warp
     ptx::mbar_init(bar(BAR_PH + 1), 4);
-    ptx::mbar_init(bar(BAR_EPI + 0), 128);
-    ptx::mbar_init(bar(BAR_EPI + 1), 128);
+    for (int i = 0; i < 8; ++i) ptx::mbar_init(bar(BAR_EPI + i), 128);
     *abort_flag = 0;
     ptx::fence_barrier_init();
     ptx::fence_proxy_async_smem();
@@ -668,13 +678,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.lse[((long long)b * p.Hq + h) * p.L + phys_q] = (m + log2f(l)) * 0.69314718055994531f;
       if (ok && staged) {
         // Staged epilogue: the gate row comes from the Q area (TMA-loaded, 64 values per
-        // 128-byte swizzled row), out = O / l * sigmoid(gate) goes to the free K/V slots
-        // in the 128-byte swizzled layout of the out map, then one thread stores by TMA.
+        // 128-byte swizzled row), out = O / l * sigmoid(gate) goes to free K/V slots in
+        // the 128-byte swizzled layout of the out map, then one thread stores by TMA.
+        // Head 0 may start while head 1's last PV still reads V, which sits in an odd
+        // slot (the producer fills K, V, K, V, ...): head 0 stages only in even slots.
+        // Output box x (32 fp32 or 64 16-bit columns, 16 KB) of head wg sits in slot
+        // 2 (x / 2) + wg, at offset (x % 2) * 16 KB.
         ptx::tc_fence_after();
         const float inv_l = 1.0f / l;
-        const uint32_t obytes = p.out_f32 ? 4u : 2u;
         const uint32_t gbase = SM_Q + (uint32_t)wg * kTileBytes;
-        const uint32_t stage = SM_SLOT + (uint32_t)wg * (uint32_t)(kTile * d) * obytes;
+        auto stage = [&](int x) {
+          return SM_SLOT + (uint32_t)(2 * (x >> 1) + wg) * kTileBytes + (uint32_t)(x & 1) * kBox;
+        };
         const uint32_t rsw = (uint32_t)(row & 7), rofs = (uint32_t)row * 128u;
         for (int j = 0; j < d / 32; ++j) {
           uint32_t o[32];
@@ -698,27 +713,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (p.out_f32) {
 #pragma unroll
             for (int v = 0; v < 8; ++v)  // box j holds columns 32j .. 32j+31
-              *reinterpret_cast<float4*>(sb + stage + (uint32_t)j * kBox + rofs + (((uint32_t)v ^ rsw) << 4)) =
+              *reinterpret_cast<float4*>(sb + stage(j) + rofs + (((uint32_t)v ^ rsw) << 4)) =
                   make_float4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
           } else {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {  // box j/2 holds columns 64(j/2) ..; piece (j%2)*4 + v
               const uint32_t q = (uint32_t)((j & 1) * 4 + v);
-              *reinterpret_cast<uint4*>(sb + stage + (uint32_t)(j >> 1) * kBox + rofs + ((q ^ rsw) << 4)) =
+              *reinterpret_cast<uint4*>(sb + stage(j >> 1) + rofs + ((q ^ rsw) << 4)) =
                   make_uint4(pack2<BF16>(y[8 * v], y[8 * v + 1]), pack2<BF16>(y[8 * v + 2], y[8 * v + 3]),
                              pack2<BF16>(y[8 * v + 4], y[8 * v + 5]), pack2<BF16>(y[8 * v + 6], y[8 * v + 7]));
             }
           }
+          // Box x (32 fp32 or 64 16-bit columns) is stored as soon as its 128 rows are
+          // staged, so the stores overlap the remaining columns' work.
+          if (p.out_f32 || (j & 1)) {
+            const int x = p.out_f32 ? j : (j >> 1);
+            ptx::fence_proxy_async_smem();  // make the rows visible to the TMA unit
+            ptx::mbar_arrive(bar(BAR_EPI + 4 * wg + x));
+            if (wq == 0 && lane == 0 && wait1(ctl, bar(BAR_EPI + 4 * wg + x), 0)) {
+              ptx::tma_store_4d(&tm.out, base + stage(x), x * (p.out_f32 ? 32 : 64), h, qrow0, b);
+              ptx::bulk_commit();
+            }
+          }
         }
-        ptx::fence_proxy_async_smem();  // make the rows visible to the TMA unit
-        ptx::mbar_arrive(bar(BAR_EPI + wg));
-        if (wq == 0 && lane == 0 && wait1(ctl, bar(BAR_EPI + wg), 0)) {
-          const int wbox = p.out_f32 ? 32 : 64;
-          for (int x = 0; x < d / wbox; ++x)
-            ptx::tma_store_4d(&tm.out, base + stage + (uint32_t)x * kBox, x * wbox, h, qrow0, b);
-          ptx::bulk_commit();
-          ptx::bulk_wait_read0();  // shared memory must outlive the store's reads
-        }
+        if (wq == 0 && lane == 0) ptx::bulk_wait_read0();  // shared memory must outlive the stores' reads
       } else if (ok) {
         ptx::tc_fence_after();
         const float inv_l = 1.0f / l;
