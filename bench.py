@@ -167,6 +167,23 @@ def make_call(case, K, bufs, ws, status):
     return launches, n_kernels
 
 
+def median_ms(fns, stream, flush, reps: int = 8, skip: int = 3) -> float:
+    """Median CUDA-event time of running `fns` in order on `stream`, L2 flushed
+    before each repetition; the first `skip` repetitions are warm-up."""
+    times = []
+    for it in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for fn in fns:
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if it >= skip:
+            times.append(a.elapsed_time(b))
+    return sorted(times)[len(times) // 2]
+
+
 def max_over_ranks(x: float, world: int, device=None) -> float:
     """The largest value of x over all ranks (timings are reported as the max)."""
     if world <= 1:
@@ -617,7 +634,30 @@ def run_ours(args, rank, world, device):
         comparisons["scanline_1mp_time_vs_dense_1mp"] = {
             "ratio": round(rec["tile_aligned"]["ms"] / ms, 4),
             "admitted_pair_ratio": round(rec["tile_aligned"]["admitted_pairs"] / (dc.seq_len ** 2), 4)}
-        del q1, k1, v1, o1, qd1, kd1, vd1, gd1
+        # The same 1 MP call on raw projections: the QK prologue as its own pass on q
+        # and k, then the core, against the prologue on k and the query half fused
+        # into the core (krea_attn_fwd_rope_q): q skips one HBM round trip.
+        table = K.rope_table(K.rope_positions(dc.text_len, dc.grid_h, dc.grid_w, device))
+        qn1, kn1 = torch.empty_like(qd1), torch.empty_like(kd1)
+        geo = dict(text_len=dc.text_len, grid_h=dc.grid_h, grid_w=dc.grid_w, out=o1, status=status)
+
+        def chained():
+            K.qk_prologue(qd1, table, out=qn1)
+            K.qk_prologue(kd1, table, out=kn1)
+            K.attention(qn1, kn1, vd1, gd1, **geo)
+
+        def fused():
+            K.qk_prologue(kd1, table, out=kn1)
+            K.attention_rope_q(qd1, kn1, vd1, gd1, table, **geo)
+
+        t_ch, t_fu = median_ms([chained], stream, flush), median_ms([fused], stream, flush)
+        comparisons["qk_prologue_fused_1mp"] = {
+            "prologue_then_attention_ms": round(t_ch, 4), "fused_q_prologue_ms": round(t_fu, 4),
+            "speedup": round(t_ch / t_fu, 4),
+            "hbm_bytes_saved": 2 * qd1.numel() * qd1.element_size(),
+            "workload": "dense 1 MP on raw q/k projections: qk_prologue(q), qk_prologue(k), attention vs "
+                        "qk_prologue(k), attention_rope_q"}
+        del q1, k1, v1, o1, qd1, kd1, vd1, gd1, qn1, kn1, table
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during the comparisons")
 

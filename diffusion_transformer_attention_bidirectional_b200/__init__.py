@@ -17,8 +17,8 @@ import torch
 from . import _lib
 from ._lib import KreaError, Params, check, lib
 
-__all__ = ["attention", "attention_backward", "quantize", "get_map", "map_size", "workspace_bytes",
-           "workspace_layout", "bwd_scratch_bytes", "make_params", "clear_cache", "KreaError"]
+__all__ = ["attention", "attention_rope_q", "attention_backward", "quantize", "get_map", "map_size",
+           "workspace_bytes", "workspace_layout", "bwd_scratch_bytes", "make_params", "clear_cache", "KreaError"]
 
 _TORCH_DT = {torch.float16: "f16", torch.bfloat16: "bf16", torch.float32: "f32"}
 
@@ -188,19 +188,8 @@ def _check_inputs(*ts):
             raise ValueError("krea attention runs on CUDA tensors only")
 
 
-def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[torch.Tensor] = None, *,
-              text_len: int, grid_h: int, grid_w: int, mode: str = "dense",
-              out: Optional[torch.Tensor] = None, out_dtype: Optional[torch.dtype] = torch.float32,
-              workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
-              stream: Optional[torch.cuda.Stream] = None, lse: Optional[torch.Tensor] = None,
-              **opts) -> torch.Tensor:
-    """out = sigmoid(gate) * softmax(scale q k^T over the admitted keys) v, per query head.
-
-    q [B, L, Hq, d], k and v [B, L, Hkv, d], gate [B, L, Hq, d] or None; L = text_len + grid_h * grid_w.
-    mode: "dense" | "tilemix" | "scanline"; `opts` are make_params keywords (q_start, q_len,
-    pattern, percentage, band_blocks, smooth_k, window, tile_aligned, text_pad, ...).
-    """
-    _check_inputs(q, k, v, gate, out, workspace, status, lse)
+def _forward_params(q, k, v, gate, out, out_dtype, workspace, status, lse, mode, text_len, grid_h, grid_w, opts):
+    """The output tensor and krea_attn_params_t of a forward call (argument marshalling)."""
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     in_dt = _TORCH_DT[q.dtype]
@@ -227,11 +216,55 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[
         p.lse = lse.data_ptr()
     if status is not None:
         p.status = status.data_ptr()
+    return out, p
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[torch.Tensor] = None, *,
+              text_len: int, grid_h: int, grid_w: int, mode: str = "dense",
+              out: Optional[torch.Tensor] = None, out_dtype: Optional[torch.dtype] = torch.float32,
+              workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None, lse: Optional[torch.Tensor] = None,
+              **opts) -> torch.Tensor:
+    """out = sigmoid(gate) * softmax(scale q k^T over the admitted keys) v, per query head.
+
+    q [B, L, Hq, d], k and v [B, L, Hkv, d], gate [B, L, Hq, d] or None; L = text_len + grid_h * grid_w.
+    mode: "dense" | "tilemix" | "scanline"; `opts` are make_params keywords (q_start, q_len,
+    pattern, percentage, band_blocks, smooth_k, window, tile_aligned, text_pad, ...).
+    """
+    _check_inputs(q, k, v, gate, out, workspace, status, lse)
+    out, p = _forward_params(q, k, v, gate, out, out_dtype, workspace, status, lse, mode, text_len, grid_h,
+                             grid_w, opts)
     rc = lib().krea_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                              gate.data_ptr() if gate is not None else None, out.data_ptr(),
                              text_len, grid_h, grid_w, _lib.MODE[mode], ctypes.byref(p),
                              _stream_ptr(stream, q.device))
     check(rc, "krea_attn_fwd")
+    return out
+
+
+def attention_rope_q(q_raw: torch.Tensor, k: torch.Tensor, v: torch.Tensor, gate: Optional[torch.Tensor],
+                     table: torch.Tensor, q_gamma: Optional[torch.Tensor] = None,
+                     rope: Optional[_lib.RopeParams] = None, *, text_len: int, grid_h: int, grid_w: int,
+                     mode: str = "dense", out: Optional[torch.Tensor] = None,
+                     out_dtype: Optional[torch.dtype] = torch.float32, status: Optional[torch.Tensor] = None,
+                     stream: Optional[torch.cuda.Stream] = None, lse: Optional[torch.Tensor] = None,
+                     **opts) -> torch.Tensor:
+    """attention(qk_prologue(q_raw, table, q_gamma), k, v, gate) in one kernel: the
+    query prologue runs on each Q tile in shared memory (krea_attn_fwd_rope_q).
+    k must already be through qk_prologue; table from rope_table with `rope`.
+    Dense and scanline modes."""
+    _check_inputs(q_raw, k, v, gate, table, q_gamma, out, status, lse)
+    d = q_raw.shape[3]
+    rope = rope if rope is not None else rope_params(d)
+    g = q_gamma.to(torch.float32).contiguous() if q_gamma is not None else None
+    out, p = _forward_params(q_raw, k, v, gate, out, out_dtype, None, status, lse, mode, text_len, grid_h,
+                             grid_w, opts)
+    rc = lib().krea_attn_fwd_rope_q(q_raw.data_ptr(), g.data_ptr() if g is not None else None, table.data_ptr(),
+                                    ctypes.byref(rope), k.data_ptr(), v.data_ptr(),
+                                    gate.data_ptr() if gate is not None else None, out.data_ptr(),
+                                    text_len, grid_h, grid_w, _lib.MODE[mode], ctypes.byref(p),
+                                    _stream_ptr(stream, q_raw.device))
+    check(rc, "krea_attn_fwd_rope_q")
     return out
 
 

@@ -104,6 +104,8 @@ SIGNATURES = {
     "krea_attn_default_params": (None, [_P, _I, _I, _I, _I, _I, _I, _I]),
     "krea_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _P, _VP]),
     "krea_attn_fwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _P, _VP]),
+    "krea_attn_fwd_rope_q": (_I, [_VP, _VP, _VP, ctypes.POINTER(RopeParams), _VP, _VP, _VP, _VP, _I, _I, _I, _I,
+                                  _P, _VP]),
     "krea_attn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _P]),
     "krea_attn_workspace_layout": (_I, [_I, _I, _I, _I, _P, ctypes.POINTER(WsLayout)]),
     "krea_attn_map_size": (_I, [_I, _I, _I, _I, _P, ctypes.POINTER(ctypes.c_int32),

@@ -71,12 +71,13 @@ constexpr int BAR_Q = 0, BAR_FULL = 1, BAR_EMPTY = BAR_FULL + kSlots, BAR_S = BA
               BAR_EPI = BAR_GATE + 1,     // 2 x 4: box x of head i staged for its TMA store (i * 4 + x)
               BAR_Q8 = BAR_EPI + 8,       // INT8 query codes landed (rows with INT8 tiles only)
               BAR_PH = BAR_Q8 + 1,        // 2: the first half of P_i (keys 0..63) written
-              N_BARS = BAR_PH + 2;
+              BAR_QN = BAR_PH + 2,        // 2: raw Q rows of head i normalised and rotated in place (q_rope)
+              N_BARS = BAR_QN + 2;
 constexpr uint32_t SM_TMEM_PTR = SM_BAR + 8 * N_BARS;
 constexpr uint32_t SM_ABORT = SM_TMEM_PTR + 4;
-constexpr uint32_t SMEM_USED = SM_BAR + 256;
+constexpr uint32_t SMEM_USED = SM_BAR + 512;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // slack to align the base to 1024 bytes
-static_assert(8 * N_BARS + 8 <= 256, "barrier block overflow");
+static_assert(8 * N_BARS + 8 <= 512, "barrier block overflow");
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 static_assert(kSlots == 4, "the staged epilogue places head 0's output in the even slots, head 1's in the odd");
 constexpr long long kDrainLimit = 4000000000LL;
@@ -243,6 +244,91 @@ __device__ __forceinline__ float i2f_exact(uint32_t x) {
   return __int_as_float((int)(x + 0x4B400000u)) - 12582912.0f;
 }
 
+// The QK prologue on one head's raw Q tile in shared memory, in place, by the
+// CTA's 256 softmax threads: RMSNorm then the 3-axis rotary turns ("Krea 2 TileMix
+// Attention (FP16/INT8 tiles)", section "What it actually patches": both run on q
+// right before the core). The work is split as krea_attn_qk_prologue splits it --
+// D / 8 lanes per row, 8 channels (16 bytes) per lane, the sum of squares as an
+// even/odd pair of fma chains per lane and then the lanes' butterfly, (x * r) *
+// gamma, the same rotation, one rounding -- with every operation an explicitly
+// rounded fp32 one, so the stored rows equal that pass's output bit for bit, and a
+// row's rotary table entries are read by its lanes as one contiguous run. Row
+// `row` of the 128-byte swizzled tile: 16-byte chunk c of the row (channels 8c ..
+// 8c+7) sits in box c / 8 at chunk (c % 8) ^ (row % 8). The tile's rows are tokens
+// qrow0 .. qrow0 + 127; rows past the sequence were zero-filled by the TMA unit
+// and stay zero.
+template <bool BF16, int D>
+struct RopeQ {
+  static constexpr int LPR = D / 8;                // lanes per row
+  static constexpr int RPW = 32 / LPR;             // rows per warp step
+  static constexpr int STEPS = kTile / (8 * RPW);  // steps of the eight warps over the 128 rows
+  int li, sub, w, pj0;
+  float4 cs[STEPS][2];  // this lane's table entries of every step: the same rows for every head
+
+  // Everything that does not depend on Q: called before Q lands, so the table
+  // loads' latency hides behind the Q copy.
+  __device__ __forceinline__ void load_table(int qrow0, int tid, const AttnDevParams& p) {
+    const int lane = tid & 31;
+    w = tid >> 5;
+    sub = lane / LPR;
+    li = lane % LPR;
+    pj0 = 4 * li;
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) {
+      const int tok = min(qrow0 + row_of(st), p.L - 1);
+      const float4* tab = reinterpret_cast<const float4*>(p.q_table + 2LL * ((long long)tok * p.q_npairs + pj0));
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2)
+        cs[st][q2] = pj0 + 2 * q2 < p.q_npairs ? __ldg(tab + q2) : make_float4(1.f, 0.f, 1.f, 0.f);
+    }
+  }
+  __device__ __forceinline__ int row_of(int st) const { return (st * 8 + w) * RPW + sub; }
+  __device__ __forceinline__ uint32_t chunk(uint32_t tile, int row) const {
+    return tile + (uint32_t)(li >> 3) * kBox + (uint32_t)row * 128u + ((((uint32_t)li & 7u) ^ ((uint32_t)row & 7u)) << 4);
+  }
+  // One head's tile, in place.
+  __device__ __forceinline__ void apply(uint32_t tile, int qrow0, const AttnDevParams& p) const {
+    float gm[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) gm[j] = p.q_gamma ? p.q_gamma[8 * li + j] : 1.0f;
+    uint4 raw[STEPS];
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) raw[st] = ptx::lds128(chunk(tile, row_of(st)));
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) {
+      const int row = row_of(st);
+      const uint16_t* e = reinterpret_cast<const uint16_t*>(&raw[st]);
+      float x[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[j] = h2f<BF16>(e[j]);
+      float se = 0.f, so = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        se = __fmaf_rn(x[2 * j], x[2 * j], se);
+        so = __fmaf_rn(x[2 * j + 1], x[2 * j + 1], so);
+      }
+      float ss = __fadd_rn(se, so);
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+      // a select for rows past the sequence (zero rows stay zero)
+      const float r = qrow0 + row < p.L ? rsqrtf(__fadd_rn(ss * (1.0f / (float)D), p.q_eps)) : 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(__fmul_rn(x[j], r), gm[j]);
+#pragma unroll
+      for (int pp = 0; pp < 4; ++pp) {  // pair pj0 + pp: (a0, a1) -> (a0 c - a1 s, a0 s + a1 c)
+        if (pj0 + pp >= p.q_npairs) break;  // channels past the rotary axes pass unturned
+        const float4 c4 = cs[st][pp >> 1];
+        const float c = (pp & 1) ? c4.z : c4.x, sn = (pp & 1) ? c4.w : c4.y;
+        const float a0 = x[2 * pp], a1 = x[2 * pp + 1];
+        x[2 * pp] = __fmaf_rn(a1, -sn, __fmul_rn(a0, c));
+        x[2 * pp + 1] = __fmaf_rn(a1, c, __fmul_rn(a0, sn));
+      }
+      ptx::sts128(chunk(tile, row), make_uint4(pack2<BF16>(x[0], x[1]), pack2<BF16>(x[2], x[3]),
+                                               pack2<BF16>(x[4], x[5]), pack2<BF16>(x[6], x[7])));
+    }
+  }
+};
+
 // Online-softmax step of one 128-key tile for one query row held by this thread.
 // v: the row of S (fp32 bits, or s32 for INT8 tiles), overwritten. mult: score
 // scale in log2 units (softmax scale * log2 e, times s_q s_k for INT8 tiles).
@@ -387,7 +473,8 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
   // the first two map entries are read before any wait, so their latency hides behind Q's
   const int ent0 = p.entries[e0];
   int e_next = n > 1 ? p.entries[e0 + 1] : 0;  // map entries are read one tile ahead
-  bool ok = wait1(ctl, bar(BAR_Q), 0);
+  // raw queries: wait for the softmax warps' prologue (which itself waited for Q)
+  bool ok = wait1(ctl, bar(p.q_rope ? BAR_QN + 0 : BAR_Q), 0);
   bool q8_ready = false;  // the INT8 query codes are awaited before the first INT8 tile
   auto need_q8 = [&](int kind) {
     if (!(kind & KREA_KIND_INT8) || q8_ready) return true;
@@ -405,7 +492,12 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
   if (ok) {
     ptx::tc_fence_after();
     const int kind0 = ent0 & 3;
-    for (int i = 0; i < nh; ++i) {
+    for (int i = 0; i < nh && ok; ++i) {
+      if (i > 0 && p.q_rope) {  // head i's Q is rotated after head 0's
+        ok = wait1(ctl, bar(BAR_QN + i), 0);
+        if (!ok) break;
+        ptx::tc_fence_after();
+      }
       qk(i, kind0, 0);
       ptx::tc_commit(bar(BAR_S + i));
     }
@@ -504,6 +596,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(bar(BAR_PH + 0), 4);  // one arrival per softmax warp
     ptx::mbar_init(bar(BAR_PH + 1), 4);
     for (int i = 0; i < 8; ++i) ptx::mbar_init(bar(BAR_EPI + i), 128);
+    ptx::mbar_init(bar(BAR_QN + 0), 256);  // one arrival per softmax thread
+    ptx::mbar_init(bar(BAR_QN + 1), 256);
     *abort_flag = 0;
     ptx::fence_barrier_init();
     ptx::fence_proxy_async_smem();
@@ -612,6 +706,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------- softmax
     ptx::regs_inc<kSoftmaxRegs>();
     const int wg = warp >> 2, wq = warp & 3;
+    bool q_ok = true;
+    if (p.q_rope) {  // the QK prologue on the raw Q tiles, head by head, all 256 threads
+      auto run = [&](auto& rq) {
+        rq.load_table(qrow0, (int)threadIdx.x, p);
+        q_ok = wait_warp(ctl, bar(BAR_Q), 0);
+        for (int i = 0; i < nh; ++i) {
+          if (q_ok) rq.apply(base + SM_Q + (uint32_t)i * kTileBytes, qrow0, p);
+          ptx::fence_proxy_async_smem();  // the rows are read by the tensor core next
+          ptx::mbar_arrive(bar(BAR_QN + i));
+        }
+      };
+      if (d == 128) {
+        RopeQ<BF16, 128> rq;
+        run(rq);
+      } else {
+        RopeQ<BF16, 64> rq;
+        run(rq);
+      }
+    }
     if (wg < nh) {
       const int h = h0 + wg;
       const int row = wq * 32 + lane;
@@ -630,8 +743,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float sq_row = p.sq ? p.sq[((long long)b * p.Hq + h) * p.nt_scale + qt] : 0.f;
       const float* sk_row = p.sk ? p.sk + ((long long)b * p.Hkv + g) * p.nt_scale : nullptr;
+      bool ok = q_ok;
       float m = kNegInf, l = 0.f;
-      bool ok = true;
       if ((p.debug_flags & 1) && wg == 0 && wq == 0) ok = wait_warp(ctl, bar(BAR_NEVER), 0);
       int e_pre = p.entries[e0];
       for (int t = 0; t < n && ok; ++t) {

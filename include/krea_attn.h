@@ -242,6 +242,32 @@ KREA_API int krea_attn_qk_prologue(const void* x, void* y, const float* gamma, c
                                    const int64_t* y_stride, const krea_rope_params_t* rope, int8_t* codes,
                                    float* scales, void* stream);
 
+/* The attention forward on RAW query projections, with the query half of the QK
+ * prologue fused into the core: each CTA normalises and rotates its Q tile in
+ * shared memory right before the first QK^T, so q makes no extra HBM round trip
+ * ("Krea 2 TileMix Attention (FP16/INT8 tiles)", section "What it actually
+ * patches": QK RMSNorm and the 3-axis RoPE run on q and k right before the core).
+ * The result equals krea_attn_qk_prologue(q_raw) followed by krea_attn_fwd bit for
+ * bit: the fused step repeats the prologue pass's arithmetic in the same order.
+ *   q_raw   [B, L, Hq, d] raw projections (layout and strides as q of krea_attn_fwd)
+ *   q_gamma d fp32 RMSNorm weights (device, 4-byte aligned) or NULL for ones
+ *   table   the rotary table of this geometry from krea_attn_rope_table (device,
+ *           16-byte aligned, row t = token t of the sequence), built with `rope`
+ *   rope    axes_dim, theta (the table's) and eps (RMSNorm)
+ *   k       keys ALREADY through the prologue (krea_attn_qk_prologue on k: each
+ *           kv head's rows are read by every query tile, so they are rotated once)
+ *   v, gate, out, text_len, grid_h, grid_w, params, stream: as krea_attn_fwd.
+ * Modes KREA_MODE_DENSE and KREA_MODE_SCANLINE; TileMix returns
+ * KREA_ERR_UNSUPPORTED (its INT8 query codes are decided on the stored prologue
+ * output: use krea_attn_qk_prologue with codes, then krea_attn_fwd). Other errors as
+ * krea_attn_fwd, and KREA_ERR_INVALID_ARG for a NULL or misaligned table, a
+ * misaligned gamma or invalid rope params. The caller owns every buffer; nothing
+ * is kept after the call. */
+KREA_API int krea_attn_fwd_rope_q(const void* q_raw, const float* q_gamma, const float* table,
+                                  const krea_rope_params_t* rope, const void* k, const void* v, const void* gate,
+                                  void* out, int text_len, int grid_h, int grid_w, int mode,
+                                  const krea_attn_params_t* params, void* stream);
+
 /* ---- sequence <-> head exchange (sequence-parallel callers) ----------------
  * A caller whose block holds the joint [text, image] sequence split by token
  * across `world` ranks (rank r: tokens [r * tokens_per_rank, (r + 1) *
