@@ -28,8 +28,10 @@ def make_params(batch: int, q_heads: int, kv_heads: int, head_dim: int, text_len
                 q_start: int = 0, q_len: int = 0, pattern: str = "band", percentage: float = 0.5,
                 band_blocks: int = 2, smooth_k: bool = True, qk_fp32_accumulate: bool = False,
                 window: int = 11, tile_aligned: bool = True, text_pad: int = 0,
-                debug_wait_limit: int = 0, debug_flags: int = 0) -> Params:
-    """krea_attn_params_t for contiguous [B, L, H, d] tensors (strides fixed up by `attention`)."""
+                debug_wait_limit: int = 0, debug_flags: int = 0, overlap_previous: bool = False) -> Params:
+    """krea_attn_params_t for contiguous [B, L, H, d] tensors (strides fixed up by `attention`).
+    overlap_previous: the call may overlap the work before it on the stream, which must write
+    nothing it reads and none of the rows it writes (e.g. the next query slice)."""
     p = Params()
     lib().krea_attn_default_params(ctypes.byref(p), batch, q_heads, kv_heads, head_dim, text_len, grid_h,
                                    grid_w)
@@ -48,6 +50,7 @@ def make_params(batch: int, q_heads: int, kv_heads: int, head_dim: int, text_len
     p.text_pad = int(text_pad)
     p.debug_wait_limit = int(debug_wait_limit)
     p.debug_flags = int(debug_flags)
+    p.overlap_previous = int(bool(overlap_previous))
     return p
 
 

@@ -10,7 +10,7 @@ from pathlib import Path
 
 LIB_PATH = Path(__file__).resolve().parent / "libkrea_attn.so"
 
-ABI_VERSION = 2
+ABI_VERSION = 3
 TILE = 128
 
 MODE = {"dense": 0, "tilemix": 1, "scanline": 2}
@@ -64,6 +64,7 @@ class Params(ctypes.Structure):
         ("debug_wait_limit", ctypes.c_int64),
         ("debug_flags", ctypes.c_int32),
         ("lse", ctypes.c_void_p),
+        ("overlap_previous", ctypes.c_int32),
     ]
 
 

@@ -391,6 +391,9 @@ int launch_forward(const void* q, const void* k, const void* v, const void* gate
   ap.wait_limit = p->debug_wait_limit > 0 ? p->debug_wait_limit : (long long)2000000000LL;
   ap.debug_flags = p->debug_flags;
   ap.lse = p->lse;
+  // no kernel of this call runs before the attention (the quantiser would): it may
+  // overlap the previous work on the stream when the caller allows it
+  ap.overlap_previous = (p->overlap_previous && !use_int8 && !centred) ? 1 : 0;
   if (q_rope) {
     ap.q_rope = 1;
     ap.q_table = q_rope->table;

@@ -565,11 +565,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Item item = decode_item((int)blockIdx.x, p);
   const int qt = item.qt, pair = item.pair, g = item.g, b = item.b;
   const int h0 = g * p.rep + pair * p.nh;
+  // Every CTA lets the next kernel on the stream launch at once: when that kernel
+  // is a programmatic dependent (the caller's overlap_previous), its CTAs take the
+  // SMs this grid's last wave leaves idle. A grid launched that way waits for its
+  // predecessor before any CTA exits, so it never completes first.
+  if (threadIdx.x == 0) ptx::launch_dependents();
   const int e0 = p.row_ptr[qt];
   const int n = p.row_ptr[qt + 1] - e0;
-  if (n <= 0) return;  // a tile of padding slots only
-  // fail fast: once any CTA of this launch (or an earlier one) has given up, do no work
-  if (p.status && *reinterpret_cast<volatile int32_t*>(p.status) != 0) return;
+  if (n <= 0 ||  // a tile of padding slots only
+      // fail fast: once any CTA of this launch (or an earlier one) has given up, do no work
+      (p.status && *reinterpret_cast<volatile int32_t*>(p.status) != 0)) {
+    if (p.overlap_previous) ptx::wait_prerequisites();
+    return;
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto bar = [&](int i) { return base + SM_BAR + 8u * (uint32_t)i; };
@@ -899,6 +907,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   if (warp == 9) ptx::tmem_dealloc(tmem, 512);
+  if (p.overlap_previous && threadIdx.x == 0) ptx::wait_prerequisites();
 }
 
 // ALL_POLY = true sends every exponential through exp2_poly2 (tests of its accuracy).
@@ -916,7 +925,17 @@ int launch(const AttnDevParams& p, const AttnMaps& maps, cudaStream_t s) {
     return KREA_ERR_CUDA;
   const long long grid = (long long)p.B * p.Hkv * p.npairs * p.n_slice_tiles;
   if (grid <= 0 || grid > 0x7fffffffLL) return KREA_ERR_INVALID_ARG;
-  attn_fwd_kernel<BF16, ALL_POLY><<<(unsigned)grid, kThreads, SMEM_ALLOC, s>>>(maps, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.overlap_previous ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, attn_fwd_kernel<BF16, ALL_POLY>, maps, p) != cudaSuccess) return KREA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? KREA_OK : KREA_ERR_CUDA;
 }
 

@@ -174,6 +174,7 @@ struct AttnDevParams {
   float* lse;          // [B, Hq, L] or null
   // q holds raw projections: the CTA applies the QK prologue to its Q tile in shared
   // memory (RMSNorm with q_gamma, then the rotary turns of q_table) before QK^T
+  int overlap_previous;  // launched as a programmatic dependent of the previous kernel on the stream
   int q_rope, q_npairs;
   float q_eps;
   const float* q_table;  // [L][q_npairs] (cos, sin)

@@ -104,6 +104,9 @@ extern "C" int krea_attn_fwd_noalloc(const void* q, const void* k, const void* v
   // krea_attn_fwd caches)
   rc = launch_build_map(g, row_ptr, entries, nullptr, nullptr, (int)(nt * nt), p->status, stream);
   if (rc != KREA_OK) return rc;
-  return launch_forward(q, k, v, gate, out, g, p, q_len, row_ptr, entries, use_int8, sc + off_ws,
+  // the attention reads the map just built on the stream: it never overlaps it
+  krea_attn_params_t pa = *p;
+  pa.overlap_previous = 0;
+  return launch_forward(q, k, v, gate, out, g, &pa, q_len, row_ptr, entries, use_int8, sc + off_ws,
                         kScratchBytes - off_ws, stream);
 }

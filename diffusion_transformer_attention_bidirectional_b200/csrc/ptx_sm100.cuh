@@ -226,6 +226,12 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   return r;
 }
 
+// ----- programmatic dependent launch -----------------------------------------
+// This CTA no longer holds back the launch of a dependent grid.
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Waits until the grids this one depends on programmatically have completed (no-op otherwise).
+__device__ __forceinline__ void wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ----- 16-byte shared-memory accesses (program order kept among them) ---------
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;

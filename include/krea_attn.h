@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define KREA_ATTN_ABI_VERSION 2
+#define KREA_ATTN_ABI_VERSION 3
 #define KREA_ATTN_TILE 128
 
 typedef enum {
@@ -122,6 +122,15 @@ typedef struct {
   float* lse;            /* optional device fp32 [B, Hq, L], 4-byte aligned: for every valid query row of the
                             slice, ln sum_j exp(softmax_scale * s_ij) over its admitted keys (the softmax
                             normaliser a backward pass needs); rows outside the slice are not written */
+  int32_t overlap_previous; /* 1: the attention kernel of this call may start while the work enqueued before
+                            it on the stream still runs (CUDA programmatic dependent launch), so its CTAs fill
+                            the SMs the previous kernel's last wave leaves idle. The caller guarantees that
+                            the earlier work writes nothing this call reads and touches none of the rows this
+                            call writes: e.g. the next query slice of the same attention ("Krea 2 TileMix
+                            Attention (FP16/INT8 tiles)": the queries are processed in slices). The call
+                            still completes after the earlier work (every CTA waits for it before it
+                            exits), so later work on the stream sees both. Ignored for TileMix, whose
+                            quantiser runs first in the same call. 0: ordinary stream order. */
 } krea_attn_params_t;
 
 /* Fill `p` with the defaults for a contiguous [B, L, H, d] layout. */
@@ -377,7 +386,8 @@ KREA_API int krea_attn_quantize(const void* q, const void* k, int text_len, int 
  * call fits up to about 1 MP; dense and scanline calls fit far beyond 4 MP). All
  * calls share the array, so calls whose GPU work overlaps (two streams, or two
  * threads on one device) race and must not be issued; calls on one stream are
- * ordered. Each call rewrites everything it reads, nothing needs clearing. The
+ * ordered (params->overlap_previous is ignored: the attention reads the map
+ * built just before it). Each call rewrites everything it reads, nothing needs clearing. The
  * first call on a device looks up the array's device address; make it before any
  * CUDA stream capture on that device. The pages describe no counterpart of this
  * entry point. */

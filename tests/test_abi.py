@@ -58,7 +58,7 @@ def test_error_strings():
     for code in range(0, -9, -1):
         s = _lib.lib().krea_attn_error_string(code).decode()
         assert s and s != "unknown error"
-    assert _lib.lib().krea_attn_abi_version() == 2
+    assert _lib.lib().krea_attn_abi_version() == 3
 
 
 def _fwd(p, T=16, H=8, W=8, mode=0, ptr=1 << 20):
