@@ -241,6 +241,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const uint32_t tS = tmem + lane_base, tP = tS + 128u, tdV = tS + 256u, tdK = tS + 384u;
     const uint32_t rsw = (uint32_t)(row & 7), rofs = (uint32_t)row * 128u;
     const int hd0 = hf * (d / 2);  // this warp's head-dim columns of dQ, dK, dV: [hd0, hd0 + d/2)
+    // Every key slot of tile j is a valid token and, with the tile-aligned rule, every
+    // valid query row of a listed query tile admits all of them: P needs no per-key
+    // predicate (padding query rows have lse = +inf, so their P is 0 anyway).
+    const int kj0 = j * kTile;
+    const bool kfull = p.tile_aligned && ((kj0 + kTile <= p.T) || (kj0 >= p.Pt && kj0 + kTile <= p.Pt + p.N));
     bool ok = true;
     for (int s = 0; s < nsteps && ok; ++s) {
       const int hh = s / n, h = g * p.rep + hh;
@@ -260,6 +265,39 @@ __global__ void __launch_bounds__(kBThreads, 1)
       ok = b_wait_warp(ctl, bar(BB_SDP), s & 1);
       if (!ok) break;
       ptx::tc_fence_after();
+      if (kfull) {  // keys 64 hf .. + 63 of S and dP -> P and dS, packed pairs, no predicate
+        uint32_t sv[64], dp[64];
+        __syncwarp();
+#pragma unroll
+        for (int ck = 0; ck < 2; ++ck) {
+          ptx::tmem_ld32(tS + 64u * hf + 32u * ck, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * ck]));
+          ptx::tmem_ld32(tP + 64u * hf + 32u * ck, *reinterpret_cast<uint32_t(*)[32]>(&dp[32 * ck]));
+        }
+        ptx::tmem_wait_ld();
+        const uint64_t sc2 = ptx::f2(p.scale_log2, p.scale_log2), nl2 = ptx::f2(-lse2, -lse2);
+        const uint64_t nd2 = ptx::f2(-Dr, -Dr);
+#pragma unroll
+        for (int pc = 0; pc < 8; ++pc) {  // 8 keys = 16 bytes of P and of dS
+          uint32_t pw[4], dw[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = 8 * pc + 2 * u;
+            float x0, x1;
+            ptx::unf2(ptx::fma2(ptx::f2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sc2, nl2), x0, x1);
+            const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+            const uint64_t pp = ptx::f2(p0, p1);
+            const uint64_t dd =
+                ptx::mul2(pp, ptx::add2(ptx::f2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nd2));
+            float d0, d1;
+            ptx::unf2(dd, d0, d1);
+            pw[u] = b_pack<BF16>(p0, p1);
+            dw[u] = b_pack<BF16>(d0, d1);
+          }
+          const uint32_t at = (uint32_t)hf * kBBox + rofs + (((uint32_t)pc ^ rsw) << 4);
+          ptx::sts128(base + BS_P + at, make_uint4(pw[0], pw[1], pw[2], pw[3]));
+          ptx::sts128(base + BS_DS + at, make_uint4(dw[0], dw[1], dw[2], dw[3]));
+        }
+      } else
       for (int ck = 0; ck < 2; ++ck) {  // keys 64 hf + 32 ck .. + 31 of S and dP -> P and dS
         uint32_t sv[32], dp[32];
         __syncwarp();
