@@ -899,6 +899,7 @@ int krea_attn_bwd(const void* q, const void* k, const void* v, const void* gate,
   if (rc == KREA_OK) rc = make_tmap(&maps.k, k, tdt, es, d, Hkv, g.L, B, p->k_stride, 64);
   if (rc == KREA_OK) rc = make_tmap(&maps.v, v, tdt, es, d, Hkv, g.L, B, p->v_stride, 64);
   if (rc == KREA_OK) rc = make_tmap(&maps.dout, dO, tdt, es, d, Hq, g.L, B, dO_stride, 64);
+  if (rc == KREA_OK) rc = make_tmap(&maps.dq, dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, Hq, g.L, B, dO_stride, 32);
   if (rc != KREA_OK) return rc;
   BwdDevParams bp;
   bp.row_ptr = map.d_row_ptr;

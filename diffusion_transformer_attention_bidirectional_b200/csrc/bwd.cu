@@ -26,7 +26,9 @@
 //   dV += P^T dO_i, dK += dS^T Q_i                  (TMEM 256..383, 384..511: the P
 //                  and dS tiles read as MN-major A operands, Q and dO as MN-major B)
 //   dQ_i part = dS K_j                              (TMEM 0..127, dS as K-major A)
-//   softmax warps add scale * dQ part into the fp32 dq buffer (vector reductions).
+//   softmax warps stage scale * dQ part in shared memory (where P and dS were) and
+//   one thread adds it into the fp32 dq buffer with TMA reduce-adds, so the
+//   additions leave the softmax warps' path.
 // Every barrier wait is bounded as in the forward kernel.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -43,10 +45,22 @@ namespace {
 
 constexpr int kBThreads = 320;
 constexpr uint32_t kBBox = 16384;        // 128 rows x 128 bytes
-constexpr uint32_t BS_K = 0, BS_V = 32768, BS_Q = 65536, BS_DO = 98304, BS_P = 131072, BS_DS = 163840;
-constexpr uint32_t BS_RED = 196608;   // 8 warps x 4 KB: dQ rows turned so a reduction covers whole rows
-constexpr uint32_t BS_BAR = BS_RED + 8 * 4096;
-enum { BB_KV = 0, BB_QF, BB_SDP, BB_PDS, BB_GRAD, BB_SFREE, BB_DRAIN, BB_QFREE, BB_N };
+// Q in two buffers (step s uses Q buffer s % 2, so the next step's Q loads while
+// this step's dK still reads its own)
+constexpr uint32_t BS_K = 0, BS_V = 32768, BS_Q = 65536, BS_DO = 131072, BS_P = 163840, BS_DS = 196608;
+// the dQ part of a step is staged for its TMA reduce-add where P and dS were (their
+// MMAs are done by then): fp32 box c (32 columns x 128 rows, 16 KB) at BS_P + c * 16 KB
+constexpr uint32_t BS_DQ = BS_P;
+constexpr uint32_t BS_BAR = BS_DS + 32768;
+enum {
+  BB_KV = 0,
+  BB_QF,           // 2: Q of a step landed in buffer s % 2
+  BB_DOF = BB_QF + 2,  // dO of a step landed
+  BB_SDP, BB_PDS, BB_GRAD, BB_SFREE, BB_DRAIN,
+  BB_QFREE,        // 2: dK of a step has read Q buffer s % 2
+  BB_DOFREE = BB_QFREE + 2,  // dV of a step has read dO
+  BB_DQ, BB_STAGED, BB_N
+};
 constexpr uint32_t BS_TMEM = BS_BAR + 8 * BB_N;
 constexpr uint32_t BS_ABORT = BS_TMEM + 4;
 constexpr uint32_t B_SMEM_ALLOC = BS_BAR + 128 + 1024;  // + slack to align the base to 1024
@@ -143,13 +157,19 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const BCtl ctl{abort_flag, p.status, p.wait_limit};
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar(BB_KV), 1);
-    ptx::mbar_init(bar(BB_QF), 1);
+    ptx::mbar_init(bar(BB_QF + 0), 1);
+    ptx::mbar_init(bar(BB_QF + 1), 1);
+    ptx::mbar_init(bar(BB_DOF), 1);
     ptx::mbar_init(bar(BB_SDP), 1);
     ptx::mbar_init(bar(BB_PDS), 8);
     ptx::mbar_init(bar(BB_GRAD), 1);
     ptx::mbar_init(bar(BB_SFREE), 8);
     ptx::mbar_init(bar(BB_DRAIN), 1);
-    ptx::mbar_init(bar(BB_QFREE), 1);
+    ptx::mbar_init(bar(BB_QFREE + 0), 1);
+    ptx::mbar_init(bar(BB_QFREE + 1), 1);
+    ptx::mbar_init(bar(BB_DOFREE), 1);
+    ptx::mbar_init(bar(BB_DQ), 8);       // every softmax warp staged its dQ rows
+    ptx::mbar_init(bar(BB_STAGED), 1);   // the staged dQ has been read by the TMA unit
     *abort_flag = 0;
     ptx::fence_barrier_init();
     ptx::fence_proxy_async_smem();
@@ -174,20 +194,28 @@ __global__ void __launch_bounds__(kBThreads, 1)
         ptx::tma_load_4d(base + BS_K + x * kBBox, &tm.k, bar(BB_KV), x * 64, g, krow0, b);
         ptx::tma_load_4d(base + BS_V + x * kBBox, &tm.v, bar(BB_KV), x * 64, g, krow0, b);
       }
-      int s = 0;
-      for (; s < nsteps; ++s) {
-        if (s > 0 && !b_wait1(ctl, bar(BB_QFREE), (s - 1) & 1)) break;  // dV, dK of s-1 read Q, dO
+      int nq = 0, nd = 0;  // Q and dO copies issued
+      for (int s = 0; s < nsteps; ++s) {
+        const uint32_t qb = (uint32_t)s & 1u;
+        // Q of step s into buffer s % 2, once dK of step s - 2 has read it
+        if (s >= 2 && !b_wait1(ctl, bar(BB_QFREE + qb), ((s >> 1) - 1) & 1)) break;
         const int h = g * p.rep + s / n;
         const int qrow0 = b_row0(p.entries[e0 + s % n] >> 2, p);
-        ptx::mbar_arrive_expect_tx(bar(BB_QF), 2 * nbox * kBBox);
-        for (int x = 0; x < nbox; ++x) {
-          ptx::tma_load_4d(base + BS_Q + x * kBBox, &tm.q, bar(BB_QF), x * 64, h, qrow0, b);
-          ptx::tma_load_4d(base + BS_DO + x * kBBox, &tm.dout, bar(BB_QF), x * 64, h, qrow0, b);
-        }
+        ptx::mbar_arrive_expect_tx(bar(BB_QF + qb), nbox * kBBox);
+        for (int x = 0; x < nbox; ++x)
+          ptx::tma_load_4d(base + BS_Q + qb * 32768u + x * kBBox, &tm.q, bar(BB_QF + qb), x * 64, h, qrow0, b);
+        ++nq;
+        // dO of step s, once dV of step s - 1 has read dO
+        if (s >= 1 && !b_wait1(ctl, bar(BB_DOFREE), (s - 1) & 1)) break;
+        ptx::mbar_arrive_expect_tx(bar(BB_DOF), nbox * kBBox);
+        for (int x = 0; x < nbox; ++x)
+          ptx::tma_load_4d(base + BS_DO + x * kBBox, &tm.dout, bar(BB_DOF), x * 64, h, qrow0, b);
+        ++nd;
       }
       // every copy this thread started lands before the CTA may exit
       b_drain(bar(BB_KV), 0);
-      if (s > 0) b_drain(bar(BB_QF), (s - 1) & 1);
+      for (int t = (nq > 2 ? nq - 2 : 0); t < nq; ++t) b_drain(bar(BB_QF + (t & 1)), (t >> 1) & 1);
+      if (nd > 0) b_drain(bar(BB_DOF), (nd - 1) & 1);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
@@ -206,13 +234,20 @@ __global__ void __launch_bounds__(kBThreads, 1)
       bool ok = b_wait1(ctl, bar(BB_KV), 0);
       if (ok) ptx::tc_fence_after();
       for (int s = 0; s < nsteps && ok; ++s) {
-        ok = b_wait1(ctl, bar(BB_QF), s & 1);
+        const uint32_t qb = (uint32_t)s & 1u, qoff = qb * (32768u >> 4);  // Q buffer of this step
+        ok = b_wait1(ctl, bar(BB_QF + qb), (s >> 1) & 1);
         if (ok && s > 0) ok = b_wait1(ctl, bar(BB_SFREE), (s - 1) & 1);  // dQ part of s-1 read out
         if (!ok) break;
         ptx::tc_fence_after();
-        for (int k = 0; k < d / 16; ++k) {  // S = Q K^T and dP = dO V^T, K = head dim
+        for (int k = 0; k < d / 16; ++k) {  // S = Q K^T, K = head dim
           const uint32_t off = (uint32_t)(k >> 2) * kb4 + (uint32_t)(k & 3) * 2u;
-          ptx::mma_f16_ss_lo(tmem, dQ_ + off, dK_ + off, ID_KK, k > 0);
+          ptx::mma_f16_ss_lo(tmem, dQ_ + qoff + off, dK_ + off, ID_KK, k > 0);
+        }
+        ok = b_wait1(ctl, bar(BB_DOF), s & 1);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        for (int k = 0; k < d / 16; ++k) {  // dP = dO V^T
+          const uint32_t off = (uint32_t)(k >> 2) * kb4 + (uint32_t)(k & 3) * 2u;
           ptx::mma_f16_ss_lo(tmem + 128u, dO_ + off, dV_ + off, ID_KK, k > 0);
         }
         ptx::tc_commit(bar(BB_SDP));
@@ -222,9 +257,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
         for (int k = 0; k < 8; ++k) {  // K = 128 query rows, 16 (2 KB of a tile) per step
           const uint32_t acc = (s > 0 || k > 0) ? 1u : 0u;
           ptx::mma_f16_ss_lo(tmem + 256u, mP + 128u * k, mDO + 128u * k, ID_MM, acc);   // dV += P^T dO
-          ptx::mma_f16_ss_lo(tmem + 384u, mDS + 128u * k, mQ + 128u * k, ID_MM, acc);   // dK += dS^T Q
         }
-        ptx::tc_commit(bar(BB_QFREE));  // Q and dO may be replaced while dQ is formed
+        ptx::tc_commit(bar(BB_DOFREE));  // the next step's dO may load
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t acc = (s > 0 || k > 0) ? 1u : 0u;
+          ptx::mma_f16_ss_lo(tmem + 384u, mDS + 128u * k, mQ + qoff + 128u * k, ID_MM, acc);  // dK += dS^T Q
+        }
+        ptx::tc_commit(bar(BB_QFREE + qb));  // this Q buffer may take step s + 2's Q
         for (int k = 0; k < 8; ++k) {  // dQ part = dS K_j, K = 128 keys
           const uint32_t off = (uint32_t)(k >> 2) * kb4 + (uint32_t)(k & 3) * 2u;
           ptx::mma_f16_ss_lo(tmem, dS_k + off, mK + 128u * k, ID_KM, k > 0);
@@ -241,6 +280,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const uint32_t tS = tmem + lane_base, tP = tS + 128u, tdV = tS + 256u, tdK = tS + 384u;
     const uint32_t rsw = (uint32_t)(row & 7), rofs = (uint32_t)row * 128u;
     const int hd0 = hf * (d / 2);  // this warp's head-dim columns of dQ, dK, dV: [hd0, hd0 + d/2)
+    const bool issuer = warp == 0 && lane == 0;  // issues the dQ reduce-adds
     // Every key slot of tile j is a valid token and, with the tile-aligned rule, every
     // valid query row of a listed query tile admits all of them: P needs no per-key
     // predicate (padding query rows have lse = +inf, so their P is 0 anyway).
@@ -265,6 +305,15 @@ __global__ void __launch_bounds__(kBThreads, 1)
       ok = b_wait_warp(ctl, bar(BB_SDP), s & 1);
       if (!ok) break;
       ptx::tc_fence_after();
+      // P and dS go where the previous step's dQ was staged: once the TMA unit read it
+      auto staged = [&]() {
+        if (s == 0) return true;
+        if (issuer) {
+          ptx::bulk_wait_read0();
+          ptx::mbar_arrive(bar(BB_STAGED));
+        }
+        return b_wait_warp(ctl, bar(BB_STAGED), (s - 1) & 1);
+      };
       if (kfull) {  // keys 64 hf .. + 63 of S and dP -> P and dS, packed pairs, no predicate
         uint32_t sv[64], dp[64];
         __syncwarp();
@@ -276,9 +325,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
         ptx::tmem_wait_ld();
         const uint64_t sc2 = ptx::f2(p.scale_log2, p.scale_log2), nl2 = ptx::f2(-lse2, -lse2);
         const uint64_t nd2 = ptx::f2(-Dr, -Dr);
+        uint32_t pw[8][4], dw[8][4];  // all of the warp's P and dS first: the exponentials
+                                      // overlap the TMA unit's read of the staged dQ
 #pragma unroll
         for (int pc = 0; pc < 8; ++pc) {  // 8 keys = 16 bytes of P and of dS
-          uint32_t pw[4], dw[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int c = 8 * pc + 2 * u;
@@ -290,14 +340,21 @@ __global__ void __launch_bounds__(kBThreads, 1)
                 ptx::mul2(pp, ptx::add2(ptx::f2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), nd2));
             float d0, d1;
             ptx::unf2(dd, d0, d1);
-            pw[u] = b_pack<BF16>(p0, p1);
-            dw[u] = b_pack<BF16>(d0, d1);
+            pw[pc][u] = b_pack<BF16>(p0, p1);
+            dw[pc][u] = b_pack<BF16>(d0, d1);
           }
-          const uint32_t at = (uint32_t)hf * kBBox + rofs + (((uint32_t)pc ^ rsw) << 4);
-          ptx::sts128(base + BS_P + at, make_uint4(pw[0], pw[1], pw[2], pw[3]));
-          ptx::sts128(base + BS_DS + at, make_uint4(dw[0], dw[1], dw[2], dw[3]));
         }
-      } else
+        ok = staged();
+        if (!ok) break;
+#pragma unroll
+        for (int pc = 0; pc < 8; ++pc) {
+          const uint32_t at = (uint32_t)hf * kBBox + rofs + (((uint32_t)pc ^ rsw) << 4);
+          ptx::sts128(base + BS_P + at, make_uint4(pw[pc][0], pw[pc][1], pw[pc][2], pw[pc][3]));
+          ptx::sts128(base + BS_DS + at, make_uint4(dw[pc][0], dw[pc][1], dw[pc][2], dw[pc][3]));
+        }
+      } else {
+      ok = staged();
+      if (!ok) break;
       for (int ck = 0; ck < 2; ++ck) {  // keys 64 hf + 32 ck .. + 31 of S and dP -> P and dS
         uint32_t sv[32], dp[32];
         __syncwarp();
@@ -329,6 +386,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
           *reinterpret_cast<uint4*>(sb + BS_DS + at) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
         }
       }
+      }
       ptx::fence_proxy_async_smem();  // the tensor core reads P and dS next
       ptx::tc_fence_before();
       __syncwarp();
@@ -336,10 +394,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
       ok = b_wait_warp(ctl, bar(BB_GRAD), s & 1);
       if (!ok) break;
       ptx::tc_fence_after();
-      // this warp's half of the dQ row into registers first, then free the TMEM
-      // columns, then add into dq: an arrive orders this thread's earlier memory
-      // operations, so the reductions come after it and the MMA thread never
-      // waits on their round trip
+      // this warp's half of the dQ row into registers, free the TMEM columns, stage
+      // it (scaled) in the 128-byte-swizzled layout of the dq map's 32-column boxes,
+      // then one thread adds the whole tile into dq by TMA. Rows of padding slots
+      // are exact zeros (their P is 0), so adding them to whatever token the box
+      // covers there changes nothing.
       uint32_t dqv[64];
       __syncwarp();
       ptx::tmem_ld32(tS + (uint32_t)hd0, *reinterpret_cast<uint32_t(*)[32]>(&dqv[0]));
@@ -348,35 +407,32 @@ __global__ void __launch_bounds__(kBThreads, 1)
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(BB_SFREE));
-      // Thread = row holds 32 consecutive floats per round; the warp's 32 x 32 block
-      // goes through a 4 KB swizzled scratch so that each reduction instruction
-      // covers 4 rows x 128 contiguous bytes (whole sectors) instead of 32 rows x
-      // 16 bytes: half the L2 atomic operations.
-      uint8_t* scr = sb + BS_RED + (uint32_t)warp * 4096u;
-      const uint32_t wsw = (uint32_t)(lane & 7);
-      const int rsub = lane >> 3, piece = lane & 7;  // read side: row 4 i + rsub, 16-byte piece
 #pragma unroll
-      for (int rnd = 0; rnd < 2; ++rnd) {  // 32 floats of the row per round (registers: constant trip)
-        if (rnd >= d / 64) break;
-        __syncwarp();
+      for (int c2 = 0; c2 < 2; ++c2) {  // boxes hd0 / 32 + c2
+        if (c2 >= d / 64) break;
+        const uint32_t box = base + BS_DQ + (uint32_t)(hd0 / 32 + c2) * kBBox;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          *reinterpret_cast<uint4*>(scr + (uint32_t)lane * 128u + (((uint32_t)k ^ wsw) << 4)) =
-              make_uint4(dqv[32 * rnd + 4 * k], dqv[32 * rnd + 4 * k + 1], dqv[32 * rnd + 4 * k + 2],
-                         dqv[32 * rnd + 4 * k + 3]);
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = 4 * i + rsub;  // row within the warp (its thread is lane rr)
-          const int pq = __shfl_sync(0xffffffffu, phys_q, rr);
-          if (pq >= 0) {
-            const uint4 u = *reinterpret_cast<const uint4*>(scr + (uint32_t)rr * 128u +
-                                                           (((uint32_t)piece ^ (uint32_t)(rr & 7)) << 4));
-            float* dst = p.dq + (((long long)b * p.L + pq) * p.Hq + h) * d + hd0 + 32 * rnd + 4 * piece;
-            red_add_v4(dst, __uint_as_float(u.x) * p.scale, __uint_as_float(u.y) * p.scale,
-                       __uint_as_float(u.z) * p.scale, __uint_as_float(u.w) * p.scale);
+        for (int v4 = 0; v4 < 8; ++v4)
+          ptx::sts128(box + rofs + (((uint32_t)v4 ^ rsw) << 4),
+                      make_uint4(__float_as_uint(__uint_as_float(dqv[32 * c2 + 4 * v4]) * p.scale),
+                                 __float_as_uint(__uint_as_float(dqv[32 * c2 + 4 * v4 + 1]) * p.scale),
+                                 __float_as_uint(__uint_as_float(dqv[32 * c2 + 4 * v4 + 2]) * p.scale),
+                                 __float_as_uint(__uint_as_float(dqv[32 * c2 + 4 * v4 + 3]) * p.scale)));
+      }
+      ptx::fence_proxy_async_smem();  // the TMA unit reads the staged rows next
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(BB_DQ));
+      if (warp == 0) {  // the issuing lane's wait decides for its whole warp
+        if (issuer) {
+          ok = b_wait1(ctl, bar(BB_DQ), s & 1);
+          if (ok) {
+            const int qrow0 = b_row0(i, p);
+            for (int c = 0; c < d / 32; ++c)
+              ptx::tma_reduce_add_4d(&tm.dq, base + BS_DQ + (uint32_t)c * kBBox, 32 * c, h, qrow0, b);
+            ptx::bulk_commit();
           }
         }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
       }
     }
     if (ok) {
@@ -405,6 +461,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
     }
   }
 
+  // every reduce-add this CTA started has finished before it exits
+  if (warp == 0 && lane == 0) ptx::bulk_wait0();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();

@@ -94,7 +94,7 @@ int launch_rope_table(const int32_t* pos, int tokens, const int axes[3], double 
 int launch_prologue(const PrologueDevParams& p, bool bf16, void* stream);
 
 // Backward (bwd.cu).
-struct alignas(64) BwdMaps { CUtensorMap q, k, v, dout; };  // dout: the dO scratch tensor
+struct alignas(64) BwdMaps { CUtensorMap q, k, v, dout, dq; };  // dout: the dO scratch tensor; dq: fp32 [B, L, Hq, d]
 struct BwdDevParams {
   const int32_t* row_ptr;
   const int32_t* entries;

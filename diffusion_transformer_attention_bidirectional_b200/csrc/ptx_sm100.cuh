@@ -85,7 +85,17 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int
       "r"(src), "r"(x), "r"(y), "r"(z), "r"(w)
       : "memory");
 }
+// shared -> global tile reduce-add (fp32 add in the memory system, bulk-group completion)
+__device__ __forceinline__ void tma_reduce_add_4d(const void* tmap, uint32_t src, int x, int y, int z, int w) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          tmap),
+      "r"(src), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// waits until every committed bulk group has completed (writes performed)
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // waits until the shared memory of every committed store group has been read
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // barrier among `count` threads on hardware barrier `id` (0 is __syncthreads)
