@@ -64,7 +64,8 @@ constexpr uint32_t SM_Q = 0;           // 2 x 32 KB
 constexpr uint32_t SM_Q8 = 65536;      // 2 x 16 KB
 constexpr uint32_t SM_SLOT = 98304;    // kSlots x 32 KB
 constexpr uint32_t SM_BAR = SM_SLOT + kSlots * kTileBytes;
-constexpr int BAR_Q = 0, BAR_FULL = 1, BAR_EMPTY = BAR_FULL + kSlots, BAR_S = BAR_EMPTY + kSlots,
+constexpr int BAR_Q = 0,  // 2: Q of head i landed
+              BAR_FULL = 2, BAR_EMPTY = BAR_FULL + kSlots, BAR_S = BAR_EMPTY + kSlots,
               BAR_P = BAR_S + 2, BAR_O = BAR_P + 2, BAR_DRAIN = BAR_O + 2, BAR_NEVER = BAR_DRAIN + 1,
               BAR_QFREE = BAR_NEVER + 1,  // the last QK^T finished: the Q area may be reused
               BAR_GATE = BAR_QFREE + 1,   // gate tiles landed in the Q area
@@ -474,7 +475,7 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
   const int ent0 = p.entries[e0];
   int e_next = n > 1 ? p.entries[e0 + 1] : 0;  // map entries are read one tile ahead
   // raw queries: wait for the softmax warps' prologue (which itself waited for Q)
-  bool ok = wait1(ctl, bar(p.q_rope ? BAR_QN + 0 : BAR_Q), 0);
+  bool ok = wait1(ctl, bar(p.q_rope ? BAR_QN + 0 : BAR_Q + 0), 0);
   bool q8_ready = false;  // the INT8 query codes are awaited before the first INT8 tile
   auto need_q8 = [&](int kind) {
     if (!(kind & KREA_KIND_INT8) || q8_ready) return true;
@@ -493,8 +494,8 @@ __device__ __forceinline__ void mma_thread(const AttnDevParams& p, uint32_t base
     ptx::tc_fence_after();
     const int kind0 = ent0 & 3;
     for (int i = 0; i < nh && ok; ++i) {
-      if (i > 0 && p.q_rope) {  // head i's Q is rotated after head 0's
-        ok = wait1(ctl, bar(BAR_QN + i), 0);
+      if (i > 0) {  // head i's Q (rotated after head 0's, with q_rope)
+        ok = wait1(ctl, bar(p.q_rope ? BAR_QN + i : BAR_Q + i), 0);
         if (!ok) break;
         ptx::tc_fence_after();
       }
@@ -586,7 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Ctl ctl{abort_flag, p.status, p.wait_limit};
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(bar(BAR_Q), 1);
+    ptx::mbar_init(bar(BAR_Q + 0), 1);
+    ptx::mbar_init(bar(BAR_Q + 1), 1);
     for (int i = 0; i < kSlots; ++i) {
       ptx::mbar_init(bar(BAR_FULL + i), 1);
       ptx::mbar_init(bar(BAR_EMPTY + i), 1);
@@ -609,6 +611,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     ptx::fence_barrier_init();
     ptx::fence_proxy_async_smem();
+    // Q goes out first, before TMEM allocation and the CTA barrier: its latency
+    // is the longest wait of a CTA's start. One barrier per head, so that head 0's
+    // QK^T may start before head 1's Q has landed.
+    const int nbox = p.d / 64, qr0 = tile_row0(qt, p);
+    for (int i = 0; i < p.nh; ++i) {
+      ptx::mbar_arrive_expect_tx(bar(BAR_Q + i), nbox * kBox);
+      for (int x = 0; x < nbox; ++x)
+        ptx::tma_load_4d(base + SM_Q + i * kTileBytes + x * kBox, &tm.q, bar(BAR_Q + i), x * 64, h0 + i, qr0, b);
+    }
   }
   if (warp == 9) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_ptr), 512);
@@ -635,14 +646,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
-      ptx::prefetch_tmap(&tm.q);
       ptx::prefetch_tmap(&tm.k);
       ptx::prefetch_tmap(&tm.v);
       const int nbox = d / 64;
-      ptx::mbar_arrive_expect_tx(bar(BAR_Q), nh * nbox * kBox);
-      for (int i = 0; i < nh; ++i)
-        for (int x = 0; x < nbox; ++x)
-          ptx::tma_load_4d(base + SM_Q + i * kTileBytes + x * kBox, &tm.q, bar(BAR_Q), x * 64, h0 + i, qrow0, b);
       if (staged && p.has_gate)  // warm L2 with the gate tiles the epilogue will need
         for (int i = 0; i < nh; ++i)
           for (int x = 0; x < nbox; ++x) ptx::tma_prefetch_l2_4d(&tm.gate, x * 64, h0 + i, qrow0, b);
@@ -684,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Every copy this thread started lands before the CTA may exit (already
       // true on the normal path, where the MMA thread consumed them all).
-      wait_drain(bar(BAR_Q), 0);
+      for (int i = 0; i < nh; ++i) wait_drain(bar(BAR_Q + i), 0);  // thread 0 issued them
       if (gate_issued) wait_drain(bar(BAR_GATE), 0);
       for (uint32_t j = (it > kSlots ? it - kSlots : 0); j < it; ++j)
         wait_drain(bar(BAR_FULL + j % kSlots), (j / kSlots) & 1);
@@ -718,8 +724,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.q_rope) {  // the QK prologue on the raw Q tiles, head by head, all 256 threads
       auto run = [&](auto& rq) {
         rq.load_table(qrow0, (int)threadIdx.x, p);
-        q_ok = wait_warp(ctl, bar(BAR_Q), 0);
         for (int i = 0; i < nh; ++i) {
+          if (q_ok) q_ok = wait_warp(ctl, bar(BAR_Q + i), 0);
           if (q_ok) rq.apply(base + SM_Q + (uint32_t)i * kTileBytes, qrow0, p);
           ptx::fence_proxy_async_smem();  // the rows are read by the tensor core next
           ptx::mbar_arrive(bar(BAR_QN + i));
