@@ -25,7 +25,11 @@
 //                  tiles (the layout TMA gives a [rows][64-element] box)
 //   dV += P^T dO_i, dK += dS^T Q_i                  (TMEM 256..383, 384..511: the P
 //                  and dS tiles read as MN-major A operands, Q and dO as MN-major B)
-//   dQ_i part = dS K_j                              (TMEM 0..127, dS as K-major A)
+//   dQ_i part = dS K_j                              (TMEM 128..255, dS as K-major A),
+//                  followed at once by the next step's S: only its dP waits for
+//                  the softmax warps to read the dQ part out
+//   P is stored and released before dS, so that dV runs while dS still waits for
+//   the TMA unit to finish reading the previous step's staged dQ in its area
 //   softmax warps stage scale * dQ part in shared memory (where P and dS were) and
 //   one thread adds it into the fp32 dq buffer with TMA reduce-adds, so the
 //   additions leave the softmax warps' path.
@@ -56,15 +60,23 @@ enum {
   BB_KV = 0,
   BB_QF,           // 2: Q of a step landed in buffer s % 2
   BB_DOF = BB_QF + 2,  // dO of a step landed
-  BB_SDP, BB_PDS, BB_GRAD, BB_SFREE, BB_DRAIN,
+  BB_SDP,
+  BB_PRDY,         // P of a step is in shared memory (dV may start)
+  BB_DSRDY,        // dS of a step is in shared memory (dK, dQ may start)
+  BB_GRAD,
+  BB_SFREE,        // the dQ part of a step has been read out of TMEM
+  BB_DRAIN,
   BB_QFREE,        // 2: dK of a step has read Q buffer s % 2
   BB_DOFREE = BB_QFREE + 2,  // dV of a step has read dO
-  BB_DQ, BB_STAGED, BB_N
+  BB_DQ,
+  BB_STAGEDP,      // the TMA unit has read the staged dQ boxes in the P area
+  BB_STAGEDDS,     // ... and those in the dS area
+  BB_N
 };
 constexpr uint32_t BS_TMEM = BS_BAR + 8 * BB_N;
 constexpr uint32_t BS_ABORT = BS_TMEM + 4;
-constexpr uint32_t B_SMEM_ALLOC = BS_BAR + 128 + 1024;  // + slack to align the base to 1024
-static_assert(BS_ABORT + 4 <= BS_BAR + 128, "barrier block");
+constexpr uint32_t B_SMEM_ALLOC = BS_BAR + 256 + 1024;  // + slack to align the base to 1024
+static_assert(BS_ABORT + 4 <= BS_BAR + 256, "barrier block");
 static_assert(B_SMEM_ALLOC <= 232448, "shared memory budget");
 constexpr long long kBDrain = 4000000000LL;
 
@@ -161,7 +173,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
     ptx::mbar_init(bar(BB_QF + 1), 1);
     ptx::mbar_init(bar(BB_DOF), 1);
     ptx::mbar_init(bar(BB_SDP), 1);
-    ptx::mbar_init(bar(BB_PDS), 8);
+    ptx::mbar_init(bar(BB_PRDY), 8);
+    ptx::mbar_init(bar(BB_DSRDY), 8);
     ptx::mbar_init(bar(BB_GRAD), 1);
     ptx::mbar_init(bar(BB_SFREE), 8);
     ptx::mbar_init(bar(BB_DRAIN), 1);
@@ -169,7 +182,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
     ptx::mbar_init(bar(BB_QFREE + 1), 1);
     ptx::mbar_init(bar(BB_DOFREE), 1);
     ptx::mbar_init(bar(BB_DQ), 8);       // every softmax warp staged its dQ rows
-    ptx::mbar_init(bar(BB_STAGED), 1);   // the staged dQ has been read by the TMA unit
+    ptx::mbar_init(bar(BB_STAGEDP), 1);  // the staged dQ has been read by the TMA unit:
+    ptx::mbar_init(bar(BB_STAGEDDS), 1); // the P area's boxes, then the dS area's
     *abort_flag = 0;
     ptx::fence_barrier_init();
     ptx::fence_proxy_async_smem();
@@ -231,19 +245,23 @@ __global__ void __launch_bounds__(kBThreads, 1)
       const uint32_t mP = ptx::sdesc_lo(base + BS_P, kBBox), mDS = ptx::sdesc_lo(base + BS_DS, kBBox);
       const uint32_t mDO = ptx::sdesc_lo(base + BS_DO, kBBox), mQ = ptx::sdesc_lo(base + BS_Q, kBBox);
       const uint32_t mK = ptx::sdesc_lo(base + BS_K, kBBox);
-      bool ok = b_wait1(ctl, bar(BB_KV), 0);
-      if (ok) ptx::tc_fence_after();
-      for (int s = 0; s < nsteps && ok; ++s) {
-        const uint32_t qb = (uint32_t)s & 1u, qoff = qb * (32768u >> 4);  // Q buffer of this step
-        ok = b_wait1(ctl, bar(BB_QF + qb), (s >> 1) & 1);
-        if (ok && s > 0) ok = b_wait1(ctl, bar(BB_SFREE), (s - 1) & 1);  // dQ part of s-1 read out
-        if (!ok) break;
-        ptx::tc_fence_after();
-        for (int k = 0; k < d / 16; ++k) {  // S = Q K^T, K = head dim
+      auto qk = [&](int s) {  // S = Q K^T of step s into columns 0..127, K = head dim
+        const uint32_t qoff = ((uint32_t)s & 1u) * (32768u >> 4);
+        for (int k = 0; k < d / 16; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * kb4 + (uint32_t)(k & 3) * 2u;
           ptx::mma_f16_ss_lo(tmem, dQ_ + qoff + off, dK_ + off, ID_KK, k > 0);
         }
-        ok = b_wait1(ctl, bar(BB_DOF), s & 1);
+      };
+      bool ok = b_wait1(ctl, bar(BB_KV), 0) && b_wait1(ctl, bar(BB_QF + 0), 0);
+      if (ok) {
+        ptx::tc_fence_after();
+        qk(0);
+      }
+      for (int s = 0; s < nsteps && ok; ++s) {
+        const uint32_t qb = (uint32_t)s & 1u, qoff = qb * (32768u >> 4);  // Q buffer of this step
+        // dP goes where the previous step's dQ part was: once the softmax warps read it
+        if (s > 0) ok = b_wait1(ctl, bar(BB_SFREE), (s - 1) & 1);
+        if (ok) ok = b_wait1(ctl, bar(BB_DOF), s & 1);
         if (!ok) break;
         ptx::tc_fence_after();
         for (int k = 0; k < d / 16; ++k) {  // dP = dO V^T
@@ -251,7 +269,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
           ptx::mma_f16_ss_lo(tmem + 128u, dO_ + off, dV_ + off, ID_KK, k > 0);
         }
         ptx::tc_commit(bar(BB_SDP));
-        ok = b_wait1(ctl, bar(BB_PDS), s & 1);
+        ok = b_wait1(ctl, bar(BB_PRDY), s & 1);
         if (!ok) break;
         ptx::tc_fence_after();
         for (int k = 0; k < 8; ++k) {  // K = 128 query rows, 16 (2 KB of a tile) per step
@@ -259,16 +277,27 @@ __global__ void __launch_bounds__(kBThreads, 1)
           ptx::mma_f16_ss_lo(tmem + 256u, mP + 128u * k, mDO + 128u * k, ID_MM, acc);   // dV += P^T dO
         }
         ptx::tc_commit(bar(BB_DOFREE));  // the next step's dO may load
+        ok = b_wait1(ctl, bar(BB_DSRDY), s & 1);  // dS lands while dV runs
+        if (!ok) break;
+        ptx::tc_fence_after();
         for (int k = 0; k < 8; ++k) {
           const uint32_t acc = (s > 0 || k > 0) ? 1u : 0u;
           ptx::mma_f16_ss_lo(tmem + 384u, mDS + 128u * k, mQ + qoff + 128u * k, ID_MM, acc);  // dK += dS^T Q
         }
         ptx::tc_commit(bar(BB_QFREE + qb));  // this Q buffer may take step s + 2's Q
-        for (int k = 0; k < 8; ++k) {  // dQ part = dS K_j, K = 128 keys
+        for (int k = 0; k < 8; ++k) {  // dQ part = dS K_j into columns 128..255, K = 128 keys
           const uint32_t off = (uint32_t)(k >> 2) * kb4 + (uint32_t)(k & 3) * 2u;
-          ptx::mma_f16_ss_lo(tmem, dS_k + off, mK + 128u * k, ID_KM, k > 0);
+          ptx::mma_f16_ss_lo(tmem + 128u, dS_k + off, mK + 128u * k, ID_KM, k > 0);
         }
         ptx::tc_commit(bar(BB_GRAD));
+        // the next step's S right behind it: S and dP of this step were consumed before
+        // its P and dS were released, and the softmax warps read the dQ part meanwhile
+        if (s + 1 < nsteps) {
+          ok = b_wait1(ctl, bar(BB_QF + (qb ^ 1u)), ((s + 1) >> 1) & 1);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          qk(s + 1);
+        }
       }
       ptx::tc_commit(bar(BB_DRAIN));
       b_drain(bar(BB_DRAIN), 0);
@@ -305,14 +334,23 @@ __global__ void __launch_bounds__(kBThreads, 1)
       ok = b_wait_warp(ctl, bar(BB_SDP), s & 1);
       if (!ok) break;
       ptx::tc_fence_after();
-      // P and dS go where the previous step's dQ was staged: once the TMA unit read it
-      auto staged = [&]() {
+      // P and dS go where the previous step's dQ was staged, each once the TMA unit
+      // has read the boxes in its area: the P area's boxes form the older bulk group
+      auto staged = [&](bool ds_area) {
         if (s == 0) return true;
         if (issuer) {
-          ptx::bulk_wait_read0();
-          ptx::mbar_arrive(bar(BB_STAGED));
+          if (ds_area || d == 64) ptx::bulk_wait_read0();
+          else ptx::bulk_wait_read1();
+          ptx::mbar_arrive(bar(ds_area ? BB_STAGEDDS : BB_STAGEDP));
         }
-        return b_wait_warp(ctl, bar(BB_STAGED), (s - 1) & 1);
+        return b_wait_warp(ctl, bar(ds_area ? BB_STAGEDDS : BB_STAGEDP), (s - 1) & 1);
+      };
+      // P first, so that dV starts while dS waits for its area
+      auto ready = [&](int bb) {
+        ptx::fence_proxy_async_smem();  // the tensor core reads the tile next
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(bb));
       };
       if (kfull) {  // keys 64 hf .. + 63 of S and dP -> P and dS, packed pairs, no predicate
         uint32_t sv[64], dp[64];
@@ -344,16 +382,24 @@ __global__ void __launch_bounds__(kBThreads, 1)
             dw[pc][u] = b_pack<BF16>(d0, d1);
           }
         }
-        ok = staged();
+        ok = staged(false);
         if (!ok) break;
 #pragma unroll
         for (int pc = 0; pc < 8; ++pc) {
           const uint32_t at = (uint32_t)hf * kBBox + rofs + (((uint32_t)pc ^ rsw) << 4);
           ptx::sts128(base + BS_P + at, make_uint4(pw[pc][0], pw[pc][1], pw[pc][2], pw[pc][3]));
+        }
+        ready(BB_PRDY);
+        ok = staged(true);
+        if (!ok) break;
+#pragma unroll
+        for (int pc = 0; pc < 8; ++pc) {
+          const uint32_t at = (uint32_t)hf * kBBox + rofs + (((uint32_t)pc ^ rsw) << 4);
           ptx::sts128(base + BS_DS + at, make_uint4(dw[pc][0], dw[pc][1], dw[pc][2], dw[pc][3]));
         }
+        ready(BB_DSRDY);
       } else {
-      ok = staged();
+      ok = staged(false) && staged(true);
       if (!ok) break;
       for (int ck = 0; ck < 2; ++ck) {  // keys 64 hf + 32 ck .. + 31 of S and dP -> P and dS
         uint32_t sv[32], dp[32];
@@ -386,11 +432,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
           *reinterpret_cast<uint4*>(sb + BS_DS + at) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
         }
       }
+      ready(BB_PRDY);
+      ready(BB_DSRDY);
       }
-      ptx::fence_proxy_async_smem();  // the tensor core reads P and dS next
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(BB_PDS));
       ok = b_wait_warp(ctl, bar(BB_GRAD), s & 1);
       if (!ok) break;
       ptx::tc_fence_after();
@@ -401,8 +445,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
       // covers there changes nothing.
       uint32_t dqv[64];
       __syncwarp();
-      ptx::tmem_ld32(tS + (uint32_t)hd0, *reinterpret_cast<uint32_t(*)[32]>(&dqv[0]));
-      if (d == 128) ptx::tmem_ld32(tS + (uint32_t)hd0 + 32u, *reinterpret_cast<uint32_t(*)[32]>(&dqv[32]));
+      ptx::tmem_ld32(tP + (uint32_t)hd0, *reinterpret_cast<uint32_t(*)[32]>(&dqv[0]));
+      if (d == 128) ptx::tmem_ld32(tP + (uint32_t)hd0 + 32u, *reinterpret_cast<uint32_t(*)[32]>(&dqv[32]));
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
@@ -427,9 +471,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
           ok = b_wait1(ctl, bar(BB_DQ), s & 1);
           if (ok) {
             const int qrow0 = b_row0(i, p);
-            for (int c = 0; c < d / 32; ++c)
+            for (int c = 0; c < d / 32; ++c) {  // boxes 0, 1 in the P area: one bulk group
               ptx::tma_reduce_add_4d(&tm.dq, base + BS_DQ + (uint32_t)c * kBBox, 32 * c, h, qrow0, b);
-            ptx::bulk_commit();
+              if (c == 1) ptx::bulk_commit();
+            }
+            if (d / 32 > 2) ptx::bulk_commit();  // boxes 2, 3 in the dS area: a second one
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
