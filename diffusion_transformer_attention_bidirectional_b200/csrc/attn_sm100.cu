@@ -571,20 +571,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   // SMs this grid's last wave leaves idle. A grid launched that way waits for its
   // predecessor before any CTA exits, so it never completes first.
   if (threadIdx.x == 0) ptx::launch_dependents();
-  const int e0 = p.row_ptr[qt];
-  const int n = p.row_ptr[qt + 1] - e0;
-  if (n <= 0 ||  // a tile of padding slots only
-      // fail fast: once any CTA of this launch (or an earlier one) has given up, do no work
-      (p.status && *reinterpret_cast<volatile int32_t*>(p.status) != 0)) {
-    if (p.overlap_previous) ptx::wait_prerequisites();
-    return;
-  }
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto bar = [&](int i) { return base + SM_BAR + 8u * (uint32_t)i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sb + SM_ABORT);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sb + SM_TMEM_PTR);
   const Ctl ctl{abort_flag, p.status, p.wait_limit};
+  // the map row and the status word are read while thread 0 sets up the barriers
+  // and starts the Q copy, which needs neither
+  const int e0 = p.row_ptr[qt];
+  const int e1 = p.row_ptr[qt + 1];
+  const int status0 = p.status ? *reinterpret_cast<volatile int32_t*>(p.status) : 0;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar(BAR_Q + 0), 1);
@@ -621,6 +617,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tma_load_4d(base + SM_Q + i * kTileBytes + x * kBox, &tm.q, bar(BAR_Q + i), x * 64, h0 + i, qr0, b);
     }
   }
+  const int n = e1 - e0;
+  if (n <= 0 ||  // a tile of padding slots only
+      // fail fast: once any CTA of this launch (or an earlier one) has given up, do no work
+      status0 != 0) {
+    if (threadIdx.x == 0)  // the Q copies land before the CTA exits
+      for (int i = 0; i < p.nh; ++i) wait_drain(bar(BAR_Q + i), 0);
+    if (p.overlap_previous) ptx::wait_prerequisites();
+    return;
+  }
+  if (threadIdx.x == 0) {
+    // the first K and V tiles follow Q at once (slots 0 and 1); the producer warp
+    // starts with the second map entry
+    const int ent0 = p.entries[e0];
+    const int nbox = p.d / 64, krow0 = tile_row0(ent0 >> 2, p);
+    const uint32_t dk0 = base + SM_SLOT, dv0 = base + SM_SLOT + kTileBytes;
+    if (ent0 & KREA_KIND_INT8) {
+      ptx::mbar_arrive_expect_tx(bar(BAR_FULL + 0), kBox);
+      ptx::tma_load_4d(dk0, &tm.k8, bar(BAR_FULL + 0), 0, g, krow0, b);
+    } else {
+      ptx::mbar_arrive_expect_tx(bar(BAR_FULL + 0), nbox * kBox);
+      for (int x = 0; x < nbox; ++x) ptx::tma_load_4d(dk0 + x * kBox, &tm.k, bar(BAR_FULL + 0), x * 64, g, krow0, b);
+    }
+    ptx::mbar_arrive_expect_tx(bar(BAR_FULL + 1), nbox * kBox);
+    for (int x = 0; x < nbox; ++x) ptx::tma_load_4d(dv0 + x * kBox, &tm.v, bar(BAR_FULL + 1), x * 64, g, krow0, b);
+  }
   if (warp == 9) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_ptr), 512);
     ptx::tmem_relinquish();
@@ -652,8 +673,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (staged && p.has_gate)  // warm L2 with the gate tiles the epilogue will need
         for (int i = 0; i < nh; ++i)
           for (int x = 0; x < nbox; ++x) ptx::tma_prefetch_l2_4d(&tm.gate, x * 64, h0 + i, qrow0, b);
-      uint32_t it = 0;
-      for (int t = 0; t < n; ++t) {
+      uint32_t it = 2;  // K and V of the first entry: issued by thread 0
+      for (int t = 1; t < n; ++t) {
         const int e = p.entries[e0 + t];
         const int krow0 = tile_row0(e >> 2, p);
         // K tile (INT8 codes for INT8 tiles)
