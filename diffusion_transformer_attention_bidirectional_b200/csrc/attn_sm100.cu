@@ -239,12 +239,6 @@ __device__ __forceinline__ void exp2_poly2(float& a, float& b) {
   b = __int_as_float(__float_as_int(p1) + (__float_as_int(j1) << 23));
 }
 
-// Exact int32 -> fp32 for |x| < 2^22 on the integer and FMA pipes (the INT8
-// tile sums are bounded by 128 * 127 * 127 < 2^21).
-__device__ __forceinline__ float i2f_exact(uint32_t x) {
-  return __int_as_float((int)(x + 0x4B400000u)) - 12582912.0f;
-}
-
 // The QK prologue on one head's raw Q tile in shared memory, in place, by the
 // CTA's 256 softmax threads: RMSNorm then the 3-axis rotary turns ("Krea 2 TileMix
 // Attention (FP16/INT8 tiles)", section "What it actually patches": both run on q
@@ -346,9 +340,13 @@ template <bool BF16, bool IS8, bool MASKED, bool ALL_POLY, bool SPLIT>
 __device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int a1, int a2, int a3, float& m,
                                              float& l, bool first, uint32_t tS, uint32_t tO, int d,
                                              uint32_t half_bar) {
+  // INT8 tiles: an s32 sum x (|x| <= 128 * 127 * 127 < 2^21) becomes the float
+  // 1.5 * 2^23 + x exactly by one integer add on its bits; the bias is taken out of the maximum below and folded
+  // into the constant of the one FMA before each exponential
+  constexpr float kBias = IS8 ? 12582912.0f : 0.0f;
 #pragma unroll
   for (int c = 0; c < 128; ++c) {
-    float r = IS8 ? i2f_exact(v[c]) : __uint_as_float(v[c]);
+    float r = IS8 ? __int_as_float((int)(v[c] + 0x4B400000u)) : __uint_as_float(v[c]);
     if constexpr (MASKED) r = ((c < a1) || (c >= a2 && c < a3)) ? r : kNegInf;
     v[c] = __float_as_uint(r);
   }
@@ -360,7 +358,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int
     mx2 = ptx::max3(mx2, __uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
     mx3 = ptx::max3(mx3, __uint_as_float(v[c + 6]), __uint_as_float(v[c + 7]));
   }
-  const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * mult;  // mult > 0
+  const float m_tile = (fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) - kBias) * mult;  // mult > 0; exact subtraction
   const float m_new = fmaxf(m, m_tile);
   if (first) {
     m = m_new;
@@ -384,7 +382,10 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&v)[128], float mult, int
     }
   }
   const float m_use = (m == kNegInf) ? 0.f : m;
-  const uint64_t mult2 = ptx::f2(mult, mult), negm2 = ptx::f2(-m_use, -m_use);
+  // (bias + x) mult - (bias mult + m) = x mult - m, the constant rounded once (INT8:
+  // an error near 2^-24 * bias * mult, ~0.75 of one code unit's weight)
+  const float c_use = IS8 ? __fmaf_rn(kBias, mult, m_use) : m_use;
+  const uint64_t mult2 = ptx::f2(mult, mult), negm2 = ptx::f2(-c_use, -c_use);
   uint64_t acc0 = ptx::f2(0.f, 0.f), acc1 = acc0;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {  // 64 keys -> 32 columns of P per half
