@@ -782,10 +782,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = q_ok;
       float m = kNegInf, l = 0.f;
       if ((p.debug_flags & 1) && wg == 0 && wq == 0) ok = wait_warp(ctl, bar(BAR_NEVER), 0);
-      int e_pre = p.entries[e0];
+      // map entries are read two tiles ahead and an INT8 tile's key-block scale one
+      // tile ahead, so that neither load waits behind the S barrier
+      auto sk_of = [&](int e) { return (sk_row && (e & KREA_KIND_INT8)) ? sk_row[e >> 2] : 0.f; };
+      int e_cur = p.entries[e0];
+      int e_nxt = n > 1 ? p.entries[e0 + 1] : 0;
+      float sk_cur = sk_of(e_cur);
       for (int t = 0; t < n && ok; ++t) {
-        const int e = e_pre;
-        if (t + 1 < n) e_pre = p.entries[e0 + t + 1];  // read one tile ahead
+        const int e = e_cur;
+        const float sk_e = sk_cur;
+        if (t + 1 < n) {
+          sk_cur = sk_of(e_nxt);
+          e_cur = e_nxt;
+        }
+        if (t + 2 < n) e_nxt = p.entries[e0 + t + 2];
         const int kb = e >> 2;
         ok = wait_warp(ctl, bar(BAR_S + wg), t & 1);
         if (!ok) break;
@@ -798,8 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kind = e & 3;
         // log2-unit score scale; INT8 tiles also carry both block scales (a zero
         // scale means an all-zero block: any positive multiplier gives score 0)
-        const float mult = (kind & KREA_KIND_INT8) ? fmaxf(p.scale_log2 * sq_row * sk_row[kb], 1e-30f)
-                                                   : p.scale_log2;
+        const float mult = (kind & KREA_KIND_INT8) ? fmaxf(p.scale_log2 * sq_row * sk_e, 1e-30f) : p.scale_log2;
         // admitted key columns of this tile: [0, a1) text, [a2, a3) image window
         const int s0 = kb * kTile;
         const int a1 = p.T - s0, a2 = klo - s0, a3 = khi - s0;
