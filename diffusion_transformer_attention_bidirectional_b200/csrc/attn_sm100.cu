@@ -17,7 +17,8 @@
 // feeds two 128 x 128 x d products. Warp roles (384 threads, 3 warpgroups):
 //   warps 0-3  softmax for head 0 (thread = query row), epilogue
 //   warps 4-7  softmax for head 1
-//   warp  8    TMA producer: Q once, then K_j, V_j into a 4-slot ring of 32 KB
+//   warp  8    TMA producer: K_j, V_j into a 4-slot ring of 32 KB (thread 0 issues
+//              Q and the first K, V right after setting up the barriers)
 //   warp  9    TMEM allocator and the single thread issuing tcgen05.mma
 //   warps 10-11 idle (they complete the third warpgroup)
 // The launch gives 168 registers per thread; the producer/MMA warpgroup drops to
