@@ -804,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t v[128];
         __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) ptx::tmem_ld32(tS + 32u * j, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * j]));
+        for (int j = 0; j < 2; ++j) ptx::tmem_ld64(tS + 64u * j, *reinterpret_cast<uint32_t(*)[64]>(&v[64 * j]));
         ptx::tmem_wait_ld();
         const int kind = e & 3;
         // log2-unit score scale; INT8 tiles also carry both block scales (a zero
