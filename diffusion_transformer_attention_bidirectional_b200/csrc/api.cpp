@@ -874,8 +874,6 @@ int krea_attn_bwd(const void* q, const void* k, const void* v, const void* gate,
   char* sc = static_cast<char*>(scratch);
   void* dO = sc;
   float* D = reinterpret_cast<float*>(sc + align256((size_t)g.L * B * Hq * d * es));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(dq, 0, (size_t)B * g.L * Hq * d * sizeof(float), s) != cudaSuccess) return KREA_ERR_CUDA;
   BwdPrepParams pp;
   pp.out = out;
   pp.dout = dout;
@@ -884,6 +882,7 @@ int krea_attn_bwd(const void* q, const void* k, const void* v, const void* gate,
   pp.dO = dO;
   pp.D = D;
   pp.dgate = gate ? dgate : nullptr;
+  pp.dq = dq;  // the prep pass zeroes dq row by row as it goes
   pp.B = B;
   pp.L = g.L;
   pp.H = Hq;

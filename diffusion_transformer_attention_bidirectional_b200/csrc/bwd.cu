@@ -573,6 +573,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepParams p) {
   for (int e = 0; e < 8; ++e) dsum = fmaf(dout[e], o[e], dsum);
   for (int off = lpr / 2; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
   if (!live) return;
+  if (p.dq) {  // dq starts from zero: the gradient kernel adds every key tile's part into it
+    float4* z = reinterpret_cast<float4*>(p.dq + rr * p.d + c0);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   uint4 w;
   uint32_t* we = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll

@@ -100,7 +100,7 @@ struct BwdDevParams {
   const int32_t* entries;
   const float* lse;     // [B, Hq, L] natural log
   const float* D;       // [B, Hq, L]
-  float* dq;            // [B, L, Hq, d] fp32, accumulated (zeroed by the host)
+  float* dq;            // [B, L, Hq, d] fp32, accumulated (zeroed by the prep pass)
   float* dk;            // [B, L, Hkv, d] fp32
   float* dv;            // [B, L, Hkv, d] fp32
   int32_t* status;
@@ -117,6 +117,7 @@ struct BwdPrepParams {
   void* dO;             // [B, L, Hq, d] input dtype, contiguous
   float* D;             // [B, Hq, L]
   float* dgate;         // [B, L, Hq, d] fp32 or null
+  float* dq;            // [B, L, Hq, d] fp32, zeroed here, or null
   int B, L, H, d;
 };
 int launch_bwd_prep(const BwdPrepParams& p, bool bf16, bool out32, void* stream);
