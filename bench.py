@@ -781,6 +781,9 @@ def _oracle_admitted_keys(ko, c, rows):
     return counts
 
 
+_SAMPLE_INPUTS = {}
+
+
 def oracle_sample(rows_per_tile: int = 4, tile_stride: int = 8):
     """Time the fp64 oracle, as it stands, on a bounded sample of the same workload:
     `rows_per_tile` query rows from every `tile_stride`-th query tile (the last
@@ -799,7 +802,10 @@ def oracle_sample(rows_per_tile: int = 4, tile_stride: int = 8):
     cases = step_cases()
     t_total, t_fixed, f_total, n_rows = 0.0, 0.0, 0.0, 0
     for c in cases:
-        q, k, v, g = S.make_inputs(c)
+        key = repr(c)  # the same seeded inputs every call: generated once per case
+        if key not in _SAMPLE_INPUTS:
+            _SAMPLE_INPUTS[key] = S.make_inputs(c)
+        q, k, v, g = _SAMPLE_INPUTS[key]
         L = c.seq_len
         nt = -(-L // TILE)
         tiles = sorted(set(range(0, nt, tile_stride)) | {nt - 1})
@@ -838,12 +844,12 @@ def run_reference(args):
     oracle_sample(rows_per_tile=1, tile_stride=64)  # untimed warm-up of numpy / BLAS
     for _ in range(args.warmup):
         oracle_sample(rows_per_tile=1, tile_stride=32)
-    runs = [oracle_sample() for _ in range(args.steps)]
+    runs = [oracle_sample(rows_per_tile=2) for _ in range(args.steps)]
     f = sum(r[0] for r in runs)
     t = sum(r[1] for r in runs)
     fixed = sum(r[2] for r in runs) / len(runs)
     value = f / t / 1e12
-    sample = (f"{runs[0][3]} query rows (4 from every 8th query tile and the last) of each variant, all 48 heads, "
+    sample = (f"{runs[0][3]} query rows (2 from every 8th query tile and the last) of each variant, all 48 heads, "
               f"batch 0, fp64 numpy oracle; time = sampled call minus a one-row one-head call, whose "
               f"whole-tensor work (map, key centring, INT8 codes) took {fixed:.2f} s per step")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
